@@ -1,0 +1,202 @@
+/*
+ * fa.h -- C ABI of the io_aware_online_b200 attention library (NVIDIA B200, sm_100a).
+ *
+ * Exact, IO-aware attention forward: O = softmax(mask(softcap(scale*Q*K^T) + ALiBi)) * V
+ * with the per-row log-sum-exp, computed by streaming K/V tiles through on-chip
+ * memory with online-softmax rescaling, so that the score matrix never reaches
+ * HBM (tag page "flash attention" (xhh.club): tiling plus online softmax, no
+ * materialised score matrix).  The argument set follows the problem statement
+ * of "FlashAttention common interfaces" (xllm-io blog), sections 3.1-3.4.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Memory: every tensor argument is a DEVICE pointer owned by the caller.  The
+ *   library allocates no memory on any call; scratch (the split-KV workspace)
+ *   is passed in.  Pointers of 16-bit tensors must be 16-byte aligned.
+ * - Execution: every call is asynchronous and stream-ordered on `stream` (a
+ *   cudaStream_t; NULL = the legacy default stream).  A nonzero return means
+ *   nothing was launched.
+ * - Dtypes: FA_FP16 or FA_BF16 for Q, K, V and O (one dtype per call); LSE,
+ *   ALiBi slopes and split partials are fp32.  fp32 inputs are not supported
+ *   (the pages: fp16/bf16 only).
+ * - Head dim: 64 or 128.
+ * - softmax_scale: a NaN means the default 1/sqrt(head_dim) (section 3.1);
+ *   otherwise it must be finite and >= 0.
+ * - Masks: the causal mask is aligned bottom-right (changelog post, v2.1): query
+ *   row i of a sequence with Sq queries and Sk keys sees key j iff
+ *   j <= i + Sk - Sq.  window_size = (left, right), -1 meaning unbounded
+ *   (section 3.1): key j is inside iff i + Sk - Sq - left <= j <= i + Sk - Sq + right.
+ *   With causal set, the causal bound limits the right side.  A row with no
+ *   allowed key gets O = 0 and LSE = -inf.
+ * - softcap > 0 replaces each scaled score s by softcap * tanh(s / softcap)
+ *   (changelog v2.6, section 5.2); 0 disables it.
+ * - alibi_slopes: NULL or fp32 [num_heads]; head h subtracts
+ *   slope[h] * |i + Sk - Sq - j| from its scores (changelog v2.4, section 5.1).
+ * - GQA/MQA: num_heads must be a multiple of num_heads_k; query head h reads
+ *   K/V head h / (num_heads / num_heads_k) (section 4.2).
+ * - Errors: functions return FA_OK (0) or an FA_ERR_* code; fa_last_error()
+ *   gives a message for the calling thread.  Faults the kernels detect on the
+ *   device (a block_table entry outside the pool, a pipeline wait that ran out
+ *   of time) set bits of a device status word, read by fa_device_status().
+ */
+#ifndef IO_AWARE_ONLINE_FA_H
+#define IO_AWARE_ONLINE_FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum fa_status {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,  /* null pointer, bad shape/stride/alignment, bad flag value */
+    FA_ERR_UNSUPPORTED = 2,  /* head_dim not in {64,128}, dtype not fp16/bf16, too many rows */
+    FA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than fa_kvcache_workspace_size() */
+    FA_ERR_CUDA = 4,         /* a CUDA runtime/driver call or kernel launch failed */
+    FA_ERR_DEVICE = 5        /* fa_device_status(): the device reported a fault */
+};
+
+enum fa_dtype { FA_FP16 = 0, FA_BF16 = 1, FA_FP32 = 2 /* fa_combine output only */ };
+
+/* Device status bits (fa_device_status). */
+enum fa_device_flag {
+    FA_DEV_WAIT_TIMEOUT = 1u,   /* a pipeline wait exceeded its time limit; that CTA stopped */
+    FA_DEV_BAD_BLOCK = 2u       /* a block_table entry was outside [0, num_blocks) */
+};
+
+/*
+ * fa_fwd -- dense or variable-length attention forward
+ * (section 3.1 flash_attn_func, section 3.2 flash_attn_varlen_func).
+ *
+ * Dense (cu_seqlens_q == cu_seqlens_k == NULL):
+ *   q [batch, seqlen_q, num_heads, head_dim], k/v [batch, seqlen_k, num_heads_k, head_dim],
+ *   out like q, lse fp32 [batch, num_heads, seqlen_q] (contiguous).
+ * Varlen (both cu_seqlens non-NULL, device int32 [batch + 1], nondecreasing, starting at 0):
+ *   q [total_q, num_heads, head_dim], k/v [total_k, num_heads_k, head_dim], out like q,
+ *   lse fp32 [num_heads, total_q].  seqlen_q / seqlen_k are then total_q / total_k
+ *   (the packed row counts, cu_seqlens_q[batch] and cu_seqlens_k[batch]) and
+ *   max_seqlen_q / max_seqlen_k bound every sequence's length.  Sequence b owns
+ *   rows cu_seqlens[b] .. cu_seqlens[b+1]-1; its mask offset is
+ *   (its key count) - (its query count).
+ * Strides: q_strides, k_strides, v_strides, o_strides are int64 [3] element strides
+ *   for (batch, seq, head); the head_dim axis must be contiguous.  NULL means the
+ *   contiguous layout above.  In varlen mode entry 0 is ignored.  Every stride must
+ *   be a multiple of 8 elements (16 bytes) and every pointer 16-byte aligned.
+ * lse may be NULL.  The N x N score matrix is never written to memory.
+ */
+FA_API int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int dtype,
+           int batch, int seqlen_q, int seqlen_k, int num_heads, int num_heads_k, int head_dim,
+           const int64_t *q_strides, const int64_t *k_strides, const int64_t *v_strides,
+           const int64_t *o_strides, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+           int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal, int window_left,
+           int window_right, float softcap, const float *alibi_slopes, void *stream);
+
+/*
+ * fa_kvcache_num_splits -- the split count fa_fwd_kvcache uses for these sizes.
+ * num_splits > 0 is returned unchanged (clamped to the number of cache pages);
+ * 0 asks for the library's heuristic, which depends only on the arguments and on
+ * the current device's SM count.  max_seqlen_k is the largest cache length
+ * (max_blocks_per_seq * page_size for a paged cache).  Returns <= 0 on bad input.
+ */
+FA_API int fa_kvcache_num_splits(int batch, int seqlen_q, int num_heads, int num_heads_k,
+                          int head_dim, int max_seqlen_k, int page_size, int num_splits);
+
+/*
+ * fa_kvcache_workspace_size -- bytes of device scratch fa_fwd_kvcache needs:
+ * splits * batch * seqlen_q * num_heads * (head_dim + 1) * 4 when the resolved split
+ * count is above 1, else 0.  Same arguments as fa_kvcache_num_splits.
+ */
+FA_API size_t fa_kvcache_workspace_size(int batch, int seqlen_q, int num_heads, int num_heads_k,
+                                 int head_dim, int max_seqlen_k, int page_size,
+                                 int num_splits);
+
+/*
+ * fa_fwd_kvcache -- attention of a few new query rows against a KV cache,
+ * split along the keys (changelog v2.2 split-KV "flash-decoding"; v2.5 paged KV
+ * cache; section 3.3 flash_attn_with_kvcache without the in-place append).
+ *
+ *   q   [batch, seqlen_q, num_heads, head_dim] contiguous; out like q;
+ *   lse fp32 [batch, num_heads, seqlen_q] or NULL.
+ * Paged cache (block_table != NULL): k_cache/v_cache are pools
+ *   [num_blocks, page_size, num_heads_k, head_dim] contiguous; block_table is
+ *   int32 [batch, max_blocks_per_seq]; entry p of sequence b names the pool block
+ *   holding its keys p*page_size .. p*page_size + page_size - 1.  page_size must be
+ *   a multiple of 64.  Entries past a sequence's last page are never read.
+ * Contiguous cache (block_table == NULL): k_cache/v_cache are
+ *   [batch, seqlen_k_max, num_heads_k, head_dim] contiguous.
+ * cache_seqlens: int32 [batch], the number of keys sequence b attends (its query
+ *   rows sit at key positions cache_seqlens[b] - seqlen_q ..).  NULL means
+ *   seqlen_k_max for every sequence (contiguous cache only).
+ * num_splits: 0 = heuristic; otherwise the keys of each sequence are cut, at
+ *   page granularity (64-token chunks for a contiguous cache), into num_splits
+ *   ranges of ceil(pages / num_splits) pages, each computed by its own CTAs, and a
+ *   second kernel combines them (fa_combine's arithmetic).  The result does not
+ *   depend on num_splits beyond rounding.
+ * workspace: device scratch of at least fa_kvcache_workspace_size(...) bytes
+ *   (may be NULL when that is 0); it holds the fp32 split partials between the
+ *   two kernels of one call, so calls that share it must be stream-ordered.
+ * Limits: num_heads / num_heads_k * seqlen_q <= 16 rows per KV head.
+ */
+FA_API int fa_fwd_kvcache(const void *q, const void *k_cache, const void *v_cache, void *out, float *lse,
+                   int dtype, int batch, int seqlen_q, int num_heads, int num_heads_k,
+                   int head_dim, const int32_t *block_table, int max_blocks_per_seq,
+                   int page_size, int num_blocks, int seqlen_k_max,
+                   const int32_t *cache_seqlens, float softmax_scale, int causal,
+                   int window_left, int window_right, float softcap,
+                   const float *alibi_slopes, int num_splits, void *workspace,
+                   size_t workspace_bytes, void *stream);
+
+/*
+ * fa_combine -- LSE-weighted combine of split partial results
+ * (section 3.4 flash_attn_combine; changelog v2.2: "an extra kernel reduces").
+ *   LSE = log sum_s exp(lse_s);  O = sum_s exp(lse_s - LSE) * O_s
+ * out_partial fp32 with logical shape [batch, seqlen, num_heads, head_dim, num_splits]
+ *   and element strides op_strides[5] (NULL = that shape, contiguous: the pages' layout);
+ * lse_partial fp32 [batch, seqlen, num_heads, num_splits], strides lp_strides[4]
+ *   (NULL = contiguous).  A split with lse_s = -inf contributes nothing (its O_s is
+ *   not read as a factor); all -inf gives O = 0, LSE = -inf.
+ * out [batch, seqlen, num_heads, head_dim] contiguous in out_dtype (FA_FP16, FA_BF16
+ *   or FA_FP32); lse fp32 [batch, num_heads, seqlen] or NULL.
+ * head_dim: any multiple of 4 up to 256 (inner loops are 16-byte vectors when the
+ *   partials are contiguous along head_dim).  num_splits: 1 .. 256.
+ */
+FA_API int fa_combine(const float *out_partial, const float *lse_partial, void *out, float *lse,
+               int out_dtype, int batch, int seqlen, int num_heads, int head_dim,
+               int num_splits, const int64_t *op_strides, const int64_t *lp_strides,
+               void *stream);
+
+/* Message describing the last error returned on the calling thread ("" if none). */
+FA_API const char *fa_last_error(void);
+
+/*
+ * fa_device_status -- synchronises the current device, then stores the OR of the
+ * FA_DEV_* bits raised by kernels since the last clear into *flags (may be NULL).
+ * clear != 0 resets them.  Returns FA_ERR_DEVICE if any bit was set, FA_OK if
+ * none, FA_ERR_CUDA if the synchronisation itself failed.
+ */
+FA_API int fa_device_status(int clear, unsigned int *flags);
+
+/*
+ * fa_set_wait_timeout_ms -- time limit of every pipeline wait inside the kernels
+ * (default 1000 ms, or the FA_WAIT_TIMEOUT_MS environment variable).  A wait that
+ * runs out sets FA_DEV_WAIT_TIMEOUT, and its CTA drains its in-flight copies and
+ * MMAs, frees its tensor memory and exits instead of hanging the GPU.  ms >= 1.
+ */
+FA_API int fa_set_wait_timeout_ms(int ms);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+FA_API int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IO_AWARE_ONLINE_FA_H */

@@ -1,0 +1,72 @@
+// fa_internal.h -- launch parameters and launcher declarations shared by the
+// host layer (fa_api.cu) and the kernel translation units.  Not installed.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+// ---------------------------------------------------------------- prefill
+struct FwdParams {
+  void* out;                       // 16-bit output rows
+  float* lse;                      // nullable
+  int64_t o_sb, o_ss, o_sh;        // output element strides (batch, seq, head)
+  const int32_t* cu_q;             // varlen offsets (NULL = dense)
+  const int32_t* cu_k;
+  int Sq, Sk;                      // dense: per-batch lengths; varlen: unused
+  int H, G;                        // query heads, query heads per KV head
+  int total_q;                     // varlen: packed query rows (LSE row stride)
+  float scale_log2;                // softmax_scale * log2(e)
+  float softcap_log2;              // softcap * log2(e)
+  float tanh_k;                    // 2 * log2(e) * softmax_scale / softcap
+  const float* alibi;              // [H] or NULL
+  int causal, wl, wr;              // mask flags; -1 = unbounded window side
+  unsigned int* status;            // device status word
+  uint64_t timeout_ns;             // bounded-wait limit
+};
+
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdParams& p, bool bf16, int d, int batch, int n_pairs,
+                       cudaStream_t stream);
+
+// ---------------------------------------------------------------- decode
+struct DecodeParams {
+  const void* q;                   // [B, Sq, H, D] contiguous
+  void* out;                       // [B, Sq, H, D] (num_splits == 1)
+  float* lse;                      // [B, H, Sq] or NULL (num_splits == 1)
+  float* ws_o;                     // [splits, B, Sq, H, D] fp32 partials (num_splits > 1)
+  float* ws_lse;                   // [splits, B, Sq, H]
+  const int32_t* block_table;      // [B, max_blocks] or NULL (contiguous cache)
+  const int32_t* cache_seqlens;    // [B] or NULL
+  int B, Sq, H, Hkv, G, R;         // R = G * Sq query rows per KV head
+  int max_blocks, page_size, num_blocks, seqlen_k_max;
+  int unit;                        // tokens per split unit (page or 64)
+  int num_splits;
+  float scale_log2, softcap_log2, tanh_k;
+  int has_softcap;
+  const float* alibi;
+  int causal, wl, wr;
+  unsigned int* status;
+  uint64_t timeout_ns;
+};
+
+cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                          bool bf16, int d, cudaStream_t stream);
+
+// ---------------------------------------------------------------- combine
+struct CombineParams {
+  const float* op;                 // partial outputs
+  const float* lp;                 // partial LSEs
+  void* out;                       // [B, S, H, D] contiguous
+  float* lse;                      // [B, H, S] or NULL
+  int64_t op_s[5];                 // b, s, h, d, split
+  int64_t lp_s[4];                 // b, s, h, split
+  int B, S, H, D, splits;
+  int out_dtype;                   // 0 fp16, 1 bf16, 2 fp32
+};
+
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+
+}  // namespace fa

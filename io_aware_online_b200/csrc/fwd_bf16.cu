@@ -1,0 +1,10 @@
+// fwd_bf16.cu -- bf16 instantiations of the prefill kernel.
+#include "fwd_launch.cuh"
+
+namespace fa {
+cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, int d, int batch, int n_pairs,
+                            cudaStream_t stream) {
+  return launch_fwd_dtype<true>(tq, tk, tv, p, d, batch, n_pairs, stream);
+}
+}  // namespace fa

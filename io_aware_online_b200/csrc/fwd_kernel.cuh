@@ -1,0 +1,436 @@
+// fwd_kernel.cuh -- exact attention forward for sm_100a (dense and varlen).
+//
+// What it computes: O = softmax(mask(softcap(scale Q K^T) + ALiBi)) V and the
+// per-row natural-log LSE, by streaming K/V blocks through shared memory with
+// online-softmax rescaling (tag page "flash attention": tiling plus online
+// softmax, the score matrix never written to HBM).  Argument semantics follow
+// "FlashAttention common interfaces" sections 3.1/3.2; the causal mask is
+// aligned bottom-right (changelog post, v2.1).
+//
+// CTA = two 128-row query tiles of one (sequence, head); 320 threads:
+//   warps 0-3  softmax warpgroup of tile 0 (thread r owns query row r = TMEM lane r)
+//   warps 4-7  softmax warpgroup of tile 1
+//   warp  8    TMA producer: Q once, then K_j / V_j blocks into a ring of stages
+//   warp  9    tensor-memory allocator and single-thread tcgen05.mma issuer
+// Tensor memory (512 columns x 128 lanes, fp32):
+//   S_t = Q_t K_j^T   at columns [128 t, 128 t + 128)        (t = 0, 1)
+//   P_t (16-bit)      aliases the first 64 columns of S_t (two values per column)
+//   O_t += P_t V_j    at columns [256 + D t, 256 + D t + D)
+// The MMA warp alternates the two tiles (ping-pong) so that the softmax of one
+// tile overlaps the tensor-core work of the other:
+//   PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1)
+// Each commit to S_t's barrier also covers the PV_t(j) issued before it, so when
+// a softmax warpgroup sees S_t(j+1) it knows P_t(j) has been consumed and O_t is
+// up to date; it may then rescale O_t in tensor memory before releasing P_t(j+1).
+// The running max is kept lazily: O is rescaled only when a row's max grows by
+// more than 8 (base-2 units); the final O / l and LSE use the same stale max, so
+// the result is unchanged.  Blocks that lie fully inside every row's allowed key
+// range skip the mask; blocks outside the CTA's key range are never loaded.
+#pragma once
+
+#include <climits>
+
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kBM = 128;          // query rows per tile
+constexpr int kBN = 128;          // keys per K/V block
+constexpr int kFwdThreads = 320;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms per row
+  static constexpr int kStages = (D == 128) ? 2 : 4;  // K and V ring depth
+  static constexpr int kTileBytes = 128 * D * 2;      // Q tile, K block or V block
+  static constexpr int kChunkBytes = 128 * 128;       // 128 rows x 128 bytes
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + 2 * kTileBytes;
+  static constexpr int kVOff = kKOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
+  // o_final[2], drain
+  static constexpr int kNumBars = 1 + 4 * kStages + 7;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;  // room to align the base to 1 KiB
+  static constexpr int kTmemCols = 512;
+  static constexpr int kOCol = 256;
+};
+
+// Wait that ignores the abort flag (used to drain this CTA's own in-flight work).
+__device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+  return true;
+}
+
+template <int D, bool BF16, bool SOFTCAP, bool ALIBI>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using Cfg = FwdCfg<D>;
+  constexpr int ST = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int h = blockIdx.x;
+  const int b = blockIdx.y;
+  const int hk = h / p.G;
+
+  // ---------------------------------------------------------- problem geometry
+  int q0 = 0, k0 = 0, Sq_b = p.Sq, Sk_b = p.Sk;
+  if (p.cu_q != nullptr) {
+    q0 = p.cu_q[b];
+    Sq_b = p.cu_q[b + 1] - q0;
+    k0 = p.cu_k[b];
+    Sk_b = p.cu_k[b + 1] - k0;
+  }
+  const int n_pairs_b = (Sq_b + 2 * kBM - 1) / (2 * kBM);
+  if (static_cast<int>(blockIdx.z) >= n_pairs_b) return;  // uniform: whole CTA leaves
+  const int pair = n_pairs_b - 1 - static_cast<int>(blockIdx.z);  // heaviest rows first
+  const int row0 = pair * 2 * kBM;
+  const int off = Sk_b - Sq_b;  // bottom-right alignment
+  const bool has_left = p.wl >= 0;
+  const bool has_right = p.causal || p.wr >= 0;
+  const int right = p.causal ? 0 : p.wr;
+  // allowed keys of row i: [lo(i), hi(i)] intersected with [0, Sk_b)
+  auto lo_of = [&](int i) { return has_left ? i + off - p.wl : INT_MIN / 2; };
+  auto hi_of = [&](int i) { return has_right ? min(i + off + right, Sk_b - 1) : Sk_b - 1; };
+  const int r_last = min(row0 + 2 * kBM - 1, Sq_b - 1);
+  const int k_begin = max(0, lo_of(row0));
+  const int k_end = hi_of(r_last) + 1;  // exclusive
+  const int j_lo = k_begin / kBN;
+  const int n_blk = (k_end > k_begin) ? (k_end + kBN - 1) / kBN - j_lo : 0;
+
+  // ---------------------------------------------------------- shared memory
+  uint8_t* sQ = smem + Cfg::kQOff;
+  uint8_t* sK = smem + Cfg::kKOff;
+  uint8_t* sV = smem + Cfg::kVOff;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 1 + ST;
+  uint64_t* v_full = bars + 1 + 2 * ST;
+  uint64_t* v_empty = bars + 1 + 3 * ST;
+  uint64_t* s_full = bars + 1 + 4 * ST;
+  uint64_t* p_full = bars + 3 + 4 * ST;
+  uint64_t* o_final = bars + 5 + 4 * ST;
+  uint64_t* drain = bars + 7 + 4 * ST;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
+
+  if (warp == 8 && lane == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full + t, 1);
+      mbar_init(p_full + t, kBM);
+      mbar_init(o_final + t, 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_holder, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+  const WaitCtx w{abort_flag, p.status, p.timeout_ns};
+  const bool varlen = p.cu_q != nullptr;
+  const int b_coord = varlen ? 0 : b;
+
+  if (warp == 8) {
+    // ======================================================== TMA producer
+    if (lane == 0 && n_blk > 0) {
+      tma_prefetch_map(&tmQ);
+      tma_prefetch_map(&tmK);
+      tma_prefetch_map(&tmV);
+      const int qrow = (varlen ? q0 : 0) + row0;
+      const int krow = varlen ? k0 : 0;
+      mbar_arrive_expect_tx(q_full, 2 * Cfg::kTileBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_4d(sQ + t * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmQ, q_full, c * 64,
+                      qrow + t * kBM, h, b_coord);
+      int last_k[ST], last_v[ST];
+      for (int s = 0; s < ST; ++s) last_k[s] = last_v[s] = -1;
+      for (int it = 0; it < n_blk; ++it) {
+        const int s = it % ST;
+        const uint32_t ph = (it / ST) & 1;
+        const int j = j_lo + it;
+        if (!wait_bounded(k_empty + s, ph ^ 1, w)) break;
+        mbar_arrive_expect_tx(k_full + s, Cfg::kTileBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_4d(sK + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmK, k_full + s, c * 64,
+                      krow + j * kBN, hk, b_coord);
+        last_k[s] = ph;
+        if (!wait_bounded(v_empty + s, ph ^ 1, w)) break;
+        mbar_arrive_expect_tx(v_full + s, Cfg::kTileBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_4d(sV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmV, v_full + s, c * 64,
+                      krow + j * kBN, hk, b_coord);
+        last_v[s] = ph;
+      }
+      if (*abort_flag) {  // let this CTA's own copies land before the smem goes away
+        wait_drain(q_full, 0, p.timeout_ns);
+        for (int s = 0; s < ST; ++s) {
+          if (last_k[s] >= 0) wait_drain(k_full + s, last_k[s], p.timeout_ns);
+          if (last_v[s] >= 0) wait_drain(v_full + s, last_v[s], p.timeout_ns);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ======================================================== MMA issuer
+    if (lane == 0 && n_blk > 0) {
+      constexpr uint32_t idesc_qk = f16_idesc(BF16, kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = f16_idesc(BF16, kBM, D, false, true);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+      // S_t = Q_t K^T: K-major A and B; step 16 of the head dim = 32 bytes inside a
+      // 128-byte swizzle atom, the next atom 16 KiB further.
+      auto qk = [&](int t, int s) {
+        const uint32_t d_tmem = tbase + t * kBM;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk / 4) * Cfg::kChunkBytes + (kk % 4) * 32;
+          mma_ss(d_tmem, sw128_desc(aQ + t * Cfg::kTileBytes + o, 16, 1024),
+                 sw128_desc(aK + s * Cfg::kTileBytes + o, 16, 1024), idesc_qk, kk > 0);
+        }
+      };
+      // O_t += P_t V: A = P from tensor memory (8 columns per 16 keys), B = V
+      // MN-major (keys advance 16 rows = 2 KiB, head-dim atoms 16 KiB apart).
+      auto pv = [&](int t, int s, bool acc) {
+        const uint32_t d_tmem = tbase + Cfg::kOCol + t * D;
+        const uint32_t a_tmem = tbase + t * kBM;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_ts(d_tmem, a_tmem + kk * 8,
+                 sw128_desc(aV + s * Cfg::kTileBytes + kk * 2048, Cfg::kChunkBytes, 1024),
+                 idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = wait_bounded(q_full, 0, w) && wait_bounded(k_full, 0, w);
+      if (ok) {
+        tc_fence_after();
+        qk(0, 0);
+        tc_commit(s_full + 0);
+        qk(1, 0);
+        tc_commit(s_full + 1);
+        tc_commit(k_empty + 0);
+        for (int it = 0; it < n_blk && ok; ++it) {
+          const int s = it % ST;
+          const uint32_t ph = (it / ST) & 1;
+          const bool more = it + 1 < n_blk;
+          const int s1 = (it + 1) % ST;
+          const uint32_t ph1 = ((it + 1) / ST) & 1;
+          if (!(ok = wait_bounded(v_full + s, ph, w))) break;
+          if (!(ok = wait_bounded(p_full + 0, it & 1, w))) break;
+          tc_fence_after();
+          pv(0, s, it > 0);
+          if (more) {
+            if (!(ok = wait_bounded(k_full + s1, ph1, w))) break;
+            tc_fence_after();
+            qk(0, s1);
+            tc_commit(s_full + 0);
+          } else {
+            tc_commit(o_final + 0);
+          }
+          if (!(ok = wait_bounded(p_full + 1, it & 1, w))) break;
+          tc_fence_after();
+          pv(1, s, it > 0);
+          tc_commit(v_empty + s);
+          if (more) {
+            qk(1, s1);
+            tc_commit(s_full + 1);
+            tc_commit(k_empty + s1);
+          } else {
+            tc_commit(o_final + 1);
+          }
+        }
+      }
+      // every MMA issued above is complete before tensor memory is released
+      tc_commit(drain);
+      wait_drain(drain, 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ======================================================== softmax warpgroups
+    const int t = warp / 4;
+    const int r = threadIdx.x % kBM;
+    const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
+    const uint32_t tS = tbase + t * kBM + lane_off;
+    const uint32_t tO = tbase + Cfg::kOCol + t * D + lane_off;
+    const int i = row0 + t * kBM + r;  // query row within the sequence
+    const int ra = row0 + t * kBM;
+    const int rb = max(ra, min(ra + kBM - 1, Sq_b - 1));
+    const int lo_i = lo_of(i), hi_i = hi_of(i);
+    const int lo_rb = lo_of(rb), hi_ra = hi_of(ra);
+    const float slope2 = ALIBI ? p.alibi[h] * kLog2e : 0.f;
+    const float ipo = static_cast<float>(i + off);
+    float m_use = -INFINITY;  // running max, base-2 units
+    float l = 0.f;            // running sum of exp2(x - m_use)
+    bool ok = true;
+
+    for (int it = 0; it < n_blk; ++it) {
+      const int kb = (j_lo + it) * kBN;
+      ok = wait_bounded(s_full + t, it & 1, w);
+      if (!__all_sync(0xffffffffu, ok)) {  // keep the warp's .sync.aligned ops uniform
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t s[kBN];
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, s + c * 32);
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) tmem_ld_wait(s + c * 32);
+
+      const bool masked = (kb < lo_rb) || (kb + kBN - 1 > hi_ra);
+      const bool plain = !SOFTCAP && !ALIBI && !masked;
+      float m_blk = -INFINITY;
+      if (plain) {
+        // scale folded into the exponent below (softmax_scale >= 0 keeps the order)
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) m_blk = fmaxf(m_blk, __uint_as_float(s[c]));
+        m_blk *= p.scale_log2;
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          float x = __uint_as_float(s[c]);
+          if constexpr (SOFTCAP) {
+            // softcap * tanh(scale * x / softcap) in base-2 units, with
+            // tanh(y) = 1 - 2 / (exp(2y) + 1)
+            const float e = ex2(x * p.tanh_k);
+            x = fmaf(-2.f * p.softcap_log2, rcp(e + 1.f), p.softcap_log2);
+          } else {
+            x *= p.scale_log2;
+          }
+          if constexpr (ALIBI) {
+            x = fmaf(-slope2, fabsf(ipo - static_cast<float>(kb + c)), x);
+          }
+          if (masked) {
+            const int kk = kb + c;
+            x = (kk >= lo_i && kk <= hi_i) ? x : -INFINITY;
+          }
+          s[c] = __float_as_uint(x);
+          m_blk = fmaxf(m_blk, x);
+        }
+      }
+      // ---- online softmax bookkeeping (lazy rescale)
+      const float m_new = fmaxf(m_use, m_blk);
+      bool need = false;
+      float alpha = 1.f;
+      if (m_use == -INFINITY) {
+        m_use = m_new;  // nothing accumulated yet: O is zero
+      } else if (m_new > m_use + kRescaleThreshold) {
+        need = true;
+        alpha = ex2(m_use - m_new);
+        m_use = m_new;
+        l *= alpha;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + c * 32, o);
+        }
+      }
+      // ---- probabilities -> 16-bit P in tensor memory (aliasing S)
+      const float factor = plain ? p.scale_log2 : 1.f;
+      const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+      float lsum = 0.f;
+#pragma unroll
+      for (int q4 = 0; q4 < kBN / 32; ++q4) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[q4 * 32 + 2 * e]), factor, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(s[q4 * 32 + 2 * e + 1]), factor, neg_m));
+          lsum += p0 + p1;
+          pk[e] = pack2<BF16>(p0, p1);
+        }
+        tmem_st16(tS + q4 * 16, pk);
+      }
+      l += lsum;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full + t);
+    }
+
+    // ---- epilogue: O / l -> 16-bit, LSE (natural log)
+    if (ok && n_blk > 0) ok = wait_bounded(o_final + t, 0, w);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const bool row_ok = i < Sq_b;
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      uint8_t* orow = nullptr;
+      if (row_ok) {
+        const int64_t ro = varlen ? static_cast<int64_t>(q0 + i) * p.o_ss
+                                  : static_cast<int64_t>(b) * p.o_sb +
+                                        static_cast<int64_t>(i) * p.o_ss;
+        orow = static_cast<uint8_t*>(p.out) + (ro + static_cast<int64_t>(h) * p.o_sh) * 2;
+      }
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (n_blk > 0) {
+          tmem_ld32(tO + c * 32, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+      if (row_ok && p.lse != nullptr) {
+        const float lse = (l > 0.f) ? (m_use + __log2f(l)) * kLn2 : -INFINITY;
+        const int64_t li = varlen ? static_cast<int64_t>(h) * p.total_q + q0 + i
+                                  : (static_cast<int64_t>(b) * p.H + h) * p.Sq + i;
+        p.lse[li] = lse;
+      }
+    }
+  }
+
+  // ---------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tbase, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace fa

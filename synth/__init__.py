@@ -21,15 +21,25 @@ import torch
 DTYPES = {"fp16": torch.float16, "bf16": torch.bfloat16}
 
 
-def _gen(seed: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+def _gen(seed: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
     g.manual_seed(int(seed))
     return g
 
 
 def randn(shape, dtype, gen: torch.Generator) -> torch.Tensor:
-    """N(0,1) fp32 draw cast to ``dtype`` (round to nearest even)."""
-    return torch.randn(*shape, generator=gen, dtype=torch.float32).to(dtype)
+    """N(0,1) fp32 draw cast to ``dtype`` (round to nearest even), on the
+    generator's device (large inputs are drawn on the GPU in chunks)."""
+    dev = gen.device
+    n = 1
+    for s in shape:
+        n *= int(s)
+    out = torch.empty(n, dtype=dtype, device=dev)
+    step = 1 << 26
+    for i in range(0, n, step):
+        m = min(step, n - i)
+        out[i:i + m] = torch.randn(m, generator=gen, dtype=torch.float32, device=dev).to(dtype)
+    return out.view(*shape)
 
 
 def dense(B, Sq, Sk, H, Hkv, d, dtype=torch.float16, seed=0):
@@ -66,7 +76,7 @@ def varlen(lengths_q, lengths_k, H, Hkv, d, dtype=torch.bfloat16, seed=0):
 
 
 def paged_cache(seqlens, page: int, Hkv: int, d: int, dtype=torch.bfloat16, seed=0,
-                tail_fill: float = float("nan"), spare_blocks: int = 0):
+                tail_fill: float = float("nan"), spare_blocks: int = 0, device="cpu"):
     """A paged KV pool for sequences of the given lengths (changelog v2.5 paged KV).
 
     Returns (kpool, vpool [num_blocks, page, Hkv, d], block_table int32 [B, max_blocks],
@@ -75,14 +85,15 @@ def paged_cache(seqlens, page: int, Hkv: int, d: int, dtype=torch.bfloat16, seed
     the ``spare_blocks`` extra blocks hold ``tail_fill`` (NaN by default) so that
     a kernel which reads them shows it.
     """
-    g = _gen(seed)
+    g = _gen(seed, device)
+    gh = _gen(seed + 7919)               # block permutation drawn on the host
     B = len(seqlens)
     nb = [(int(L) + page - 1) // page for L in seqlens]
     total = sum(nb) + int(spare_blocks)
     max_blocks = max(1, max(nb) if nb else 1)
     kpool = randn((total, page, Hkv, d), dtype, g)
     vpool = randn((total, page, Hkv, d), dtype, g)
-    perm = torch.randperm(total, generator=g).to(torch.int32)
+    perm = torch.randperm(total, generator=gh).to(torch.int32)
     bt = torch.full((B, max_blocks), -1, dtype=torch.int32)
     used = torch.zeros(total, dtype=torch.bool)
     pos = 0
@@ -96,8 +107,9 @@ def paged_cache(seqlens, page: int, Hkv: int, d: int, dtype=torch.bfloat16, seed
             if valid < page:
                 kpool[blk, valid:] = tail_fill
                 vpool[blk, valid:] = tail_fill
-    kpool[~used] = tail_fill
-    vpool[~used] = tail_fill
+    unused = (~used).nonzero().flatten().to(kpool.device)
+    kpool[unused] = tail_fill
+    vpool[unused] = tail_fill
     return kpool, vpool, bt, torch.tensor([int(L) for L in seqlens], dtype=torch.int32)
 
 

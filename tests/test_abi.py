@@ -1,0 +1,134 @@
+"""C-ABI checks that need no GPU: the library builds, loads and exports every
+symbol include/fa.h declares, and argument validation returns the documented
+error codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import io_aware_online_b200 as fa
+from io_aware_online_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE = 0, 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return fa.load()
+
+
+def header_symbols():
+    src = open(os.path.join(ROOT, "include", "fa.h")).read()
+    return re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", src)
+
+
+def test_header_declares_the_entry_points():
+    names = set(header_symbols())
+    assert {"fa_fwd", "fa_fwd_kvcache", "fa_combine", "fa_kvcache_workspace_size",
+            "fa_kvcache_num_splits", "fa_last_error", "fa_device_status"} <= names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_symbols():
+        assert hasattr(lib, name), f"{name} not exported"
+
+
+def test_version_and_error_string(lib):
+    assert lib.fa_version() >= 100
+    assert isinstance(lib.fa_last_error(), bytes)
+
+
+# fake, 16-byte aligned "device" pointers: validation rejects before any device use
+P = ctypes.c_void_p(0x10000)
+MIS = ctypes.c_void_p(0x10008)
+
+
+def fwd(lib, **kw):
+    a = dict(q=P, k=P, v=P, out=P, lse=None, dtype=0, B=1, Sq=128, Sk=128, H=2, Hkv=2, d=64,
+             qs=None, ks=None, vs=None, os_=None, cuq=None, cuk=None, mq=0, mk=0,
+             scale=float("nan"), causal=0, wl=-1, wr=-1, softcap=0.0, alibi=None, stream=None)
+    a.update(kw)
+    return lib.fa_fwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["dtype"], a["B"], a["Sq"],
+                      a["Sk"], a["H"], a["Hkv"], a["d"], a["qs"], a["ks"], a["vs"], a["os_"],
+                      a["cuq"], a["cuk"], a["mq"], a["mk"], a["scale"], a["causal"], a["wl"],
+                      a["wr"], a["softcap"], a["alibi"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), FA_ERR_UNSUPPORTED),
+    (dict(dtype=2), FA_ERR_UNSUPPORTED),
+    (dict(H=3, Hkv=2), FA_ERR_INVALID_ARG),
+    (dict(Hkv=0), FA_ERR_INVALID_ARG),
+    (dict(q=None), FA_ERR_INVALID_ARG),
+    (dict(k=MIS), FA_ERR_INVALID_ARG),
+    (dict(wl=-2), FA_ERR_INVALID_ARG),
+    (dict(wr=-5), FA_ERR_INVALID_ARG),
+    (dict(softcap=-1.0), FA_ERR_INVALID_ARG),
+    (dict(softcap=float("inf")), FA_ERR_INVALID_ARG),
+    (dict(scale=-0.5), FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), FA_ERR_INVALID_ARG),
+    (dict(Sq=-1), FA_ERR_INVALID_ARG),
+    (dict(cuq=P), FA_ERR_INVALID_ARG),                       # varlen needs both offsets
+    (dict(cuq=P, cuk=P, mq=300, mk=10), FA_ERR_INVALID_ARG),  # max_seqlen beyond total rows
+])
+def test_fwd_validation(lib, kw, code):
+    assert fwd(lib, **kw) == code
+    assert lib.fa_last_error()
+
+
+def test_fwd_bad_strides(lib):
+    bad = (ctypes.c_int64 * 3)(128 * 2 * 64, 2 * 64, 60)     # head stride not a multiple of 8
+    assert fwd(lib, qs=bad) == FA_ERR_INVALID_ARG
+
+
+def test_fwd_empty_is_a_noop(lib):
+    assert fwd(lib, B=0) == FA_OK
+    assert fwd(lib, Sq=0) == FA_OK
+
+
+def kvc(lib, **kw):
+    a = dict(q=P, kc=P, vc=P, out=P, lse=None, dtype=1, B=2, Sq=1, H=32, Hkv=8, d=128, bt=P,
+             maxb=4, page=256, nblk=8, skmax=0, cs=P, scale=float("nan"), causal=1, wl=-1,
+             wr=-1, softcap=0.0, alibi=None, splits=1, ws=None, wsb=0, stream=None)
+    a.update(kw)
+    return lib.fa_fwd_kvcache(a["q"], a["kc"], a["vc"], a["out"], a["lse"], a["dtype"], a["B"],
+                              a["Sq"], a["H"], a["Hkv"], a["d"], a["bt"], a["maxb"], a["page"],
+                              a["nblk"], a["skmax"], a["cs"], a["scale"], a["causal"], a["wl"],
+                              a["wr"], a["softcap"], a["alibi"], a["splits"], a["ws"], a["wsb"],
+                              a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(page=100), FA_ERR_INVALID_ARG),
+    (dict(cs=None), FA_ERR_INVALID_ARG),            # paged cache needs cache_seqlens
+    (dict(Sq=5), FA_ERR_UNSUPPORTED),               # 4 * 5 = 20 rows per KV head > 16
+    (dict(nblk=0), FA_ERR_INVALID_ARG),
+    (dict(d=80), FA_ERR_UNSUPPORTED),
+    (dict(splits=4, ws=None, wsb=0), FA_ERR_WORKSPACE),
+    (dict(bt=None, skmax=-1), FA_ERR_INVALID_ARG),
+])
+def test_kvcache_validation(lib, kw, code):
+    assert kvc(lib, **kw) == code
+
+
+def test_splits_and_workspace_size(lib):
+    # explicit split counts are clamped to the number of pages
+    assert lib.fa_kvcache_num_splits(64, 1, 32, 8, 128, 32768, 256, 16) == 16
+    assert lib.fa_kvcache_num_splits(64, 1, 32, 8, 128, 512, 256, 16) == 2
+    assert lib.fa_kvcache_workspace_size(64, 1, 32, 8, 128, 32768, 256, 1) == 0
+    assert lib.fa_kvcache_workspace_size(64, 1, 32, 8, 128, 32768, 256, 4) == 4 * 64 * 32 * 129 * 4
+
+
+def test_combine_validation(lib):
+    assert lib.fa_combine(P, P, P, None, 0, 1, 1, 1, 64, 0, None, None, None) == FA_ERR_INVALID_ARG
+    assert lib.fa_combine(P, P, P, None, 0, 1, 1, 1, 64, 300, None, None, None) == FA_ERR_INVALID_ARG
+    assert lib.fa_combine(P, P, P, None, 7, 1, 1, 1, 64, 2, None, None, None) == FA_ERR_UNSUPPORTED
+    assert lib.fa_combine(P, P, P, None, 0, 1, 1, 1, 62, 2, None, None, None) == FA_ERR_INVALID_ARG
+
+
+def test_timeout_setter(lib):
+    assert lib.fa_set_wait_timeout_ms(0) == FA_ERR_INVALID_ARG
+    assert lib.fa_set_wait_timeout_ms(1000) == FA_OK
