@@ -1,0 +1,391 @@
+"""Benchmark of the attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  1. prefill forward (fa_fwd): causal, B=4, S=4096, H=32, d=64, fp16
+  2. paged split-KV decode (fa_fwd_kvcache) + LSE combine: B=64, Sq=1, H=32,
+     Hkv=8, d=128, bf16, cache lengths U{1K..32K}, pages of 256, random
+     block_table, num_splits (default 16)
+Reported: ``value`` = prefill TFLOPS (4*d*sum of allowed (i, j) pairs / time);
+``decode`` = KV-cache GB/s (valid cache bytes + q/out/lse/block_table / time).
+Both are also given as fractions of the measured B200 peaks.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+       [--num-splits S] [--no-cpu-baseline] [--no-e2e]
+For N > 1 launch under torch.distributed.run; every rank runs an independent
+replica on its own seeded data (weak scaling, no collective on the data path);
+the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+PREFILL = dict(B=4, S=4096, H=32, Hkv=32, d=64, dtype="fp16", causal=True)
+DECODE = dict(B=64, Sq=1, H=32, Hkv=8, d=128, dtype="bf16", lo=1024, hi=32768, page=256)
+METRIC = "attn fwd TFLOPS (causal prefill) & decode KV GB/s, % of B200 roofline"
+
+
+def causal_pairs(Sq: int, Sk: int) -> int:
+    """Number of allowed (i, j) pairs of a bottom-right causal mask: row i sees
+    keys 0 .. i + Sk - Sq."""
+    off = Sk - Sq
+    return sum(min(Sk, max(0, i + off + 1)) for i in range(Sq))
+
+
+def prefill_flops(c=PREFILL) -> float:
+    return 4.0 * c["d"] * c["B"] * c["H"] * causal_pairs(c["S"], c["S"])
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk["hbm_gbs"], pk["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"]}
+        busy = [m for m in mhz if m > 0.5 * max(mhz)] or mhz
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+def dist_setup(gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != gpus:
+        if world > 1 or gpus > 1:
+            raise SystemExit(f"--gpus {gpus} but WORLD_SIZE={world}: launch with torch.distributed.run")
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- workloads
+def make_prefill(rank, dev):
+    c = PREFILL
+    dt = synth.DTYPES[c["dtype"]]
+    q, k, v = synth.dense(c["B"], c["S"], c["S"], c["H"], c["Hkv"], c["d"], dt,
+                          seed=1003 + 100 * rank)
+    return q, k, v
+
+
+def make_decode(rank, dev):
+    c = DECODE
+    dt = synth.DTYPES[c["dtype"]]
+    lens = synth.varlen_lengths(c["B"], c["lo"], c["hi"], seed=1005 + 100 * rank)
+    kp, vp, bt, cs = synth.paged_cache(lens, c["page"], c["Hkv"], c["d"], dt,
+                                       seed=1005 + 100 * rank, device=dev)
+    q = synth.randn((c["B"], c["Sq"], c["H"], c["d"]), dt,
+                    torch.Generator().manual_seed(1006 + 100 * rank))
+    return q, kp, vp, bt, cs, lens
+
+
+def decode_bytes(lens, splits):
+    c = DECODE
+    kv = sum(lens) * c["Hkv"] * c["d"] * 2 * 2               # K and V, valid tokens only
+    io = c["B"] * c["Sq"] * c["H"] * c["d"] * 2 * 2          # q in, out
+    io += c["B"] * c["H"] * c["Sq"] * 4                       # lse
+    bt = sum((L + c["page"] - 1) // c["page"] for L in lens) * 4 + c["B"] * 4
+    return kv + io + bt
+
+
+def run_ours(args, rank, world, local):
+    import io_aware_online_b200 as fa
+    from io_aware_online_b200 import build as fa_build
+    fa_build.build()
+    fa.load()
+    dev = torch.device("cuda", local)
+    hbm_peak, tflops_peak, peak_src = load_peaks()
+
+    q, k, v = make_prefill(rank, dev)
+    qd_, kd_, vd_ = q.to(dev), k.to(dev), v.to(dev)
+    out_p = torch.empty_like(qd_)
+    lse_p = torch.empty((PREFILL["B"], PREFILL["H"], PREFILL["S"]), dtype=torch.float32, device=dev)
+    dq, kp, vp, bt, cs, lens = make_decode(rank, dev)
+    dq_d, bt_d, cs_d = dq.to(dev), bt.to(dev), cs.to(dev)
+    splits = args.num_splits
+    c = DECODE
+    ws_bytes = fa.fa_kvcache_workspace_size(c["B"], c["Sq"], c["H"], c["Hkv"], c["d"],
+                                            bt.shape[1] * c["page"], c["page"], splits)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    out_d = torch.empty_like(dq_d)
+    lse_d = torch.empty((c["B"], c["H"], c["Sq"]), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+
+    def prefill():
+        fa.fa_fwd(qd_, kd_, vd_, out=out_p, lse=lse_p, causal=True, stream=stream)
+
+    def decode():
+        fa.fa_fwd_kvcache(dq_d, kp, vp, cache_seqlens=cs_d, block_table=bt_d, causal=True,
+                          num_splits=splits, out=out_d, lse=lse_d, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        prefill()
+        decode()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with Clocks(dev.index if dev.index is not None else 0) as clk:
+        for s in range(K):
+            flush.zero_()                       # L2 flushed between steps (not timed)
+            ev[s][0].record(stream)
+            prefill()
+            ev[s][1].record(stream)
+            decode()
+            ev[s][2].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    t_pre = sum(e[0].elapsed_time(e[1]) for e in ev) / K      # ms per launch
+    t_dec = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    t_step = t_pre + t_dec
+    t_pre_max = max_over_ranks(t_pre, world)
+    t_dec_max = max_over_ranks(t_dec, world)
+    t_step_max = max_over_ranks(t_step, world)
+    assert fa.fa_device_status(clear=True) == 0, "device status flags raised during the bench"
+
+    flops = prefill_flops()
+    tflops = flops / (t_pre_max * 1e-3) / 1e12 * world
+    dbytes = decode_bytes(lens, splits)
+    gbs = dbytes / (t_dec_max * 1e-3) / 1e9 * world
+    res = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(t_step_max, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp16 (prefill), bf16 (decode); fp32 accumulate",
+        "data": "synthetic (seeded N(0,1))",
+        "config": {
+            "workload": "causal prefill B=4 S=4096 H=32 d=64 fp16 + paged split-KV decode "
+                        "B=64 H=32 Hkv=8 d=128 bf16 cache U{1K..32K} page 256",
+            "prefill": dict(PREFILL, ms=round(t_pre_max, 4), flop=flops),
+            "decode": dict(DECODE, num_splits=splits, sum_cache_tokens=int(sum(lens)),
+                           ms=round(t_dec_max, 4), bytes=dbytes),
+            "l2": "flushed between steps (256 MiB write, untimed)",
+            "parallelism": f"dp{world} (independent replicas)",
+        },
+        "decode": {
+            "value": round(gbs, 1), "unit": "GB/s", "ms": round(t_dec_max, 4),
+            "roofline": {"bound": "hbm", "achieved": round(dbytes / (t_dec_max * 1e-3) / 1e9, 1),
+                         "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(dbytes / (t_dec_max * 1e-3) / 1e9 / hbm_peak, 4),
+                         "traffic": None, "peak_source": peak_src},
+        },
+        "roofline": {"bound": "tensor", "achieved": round(flops / (t_pre * 1e-3) / 1e12, 2),
+                     "peak": tflops_peak, "unit": "TFLOP/s",
+                     "frac": round(flops / (t_pre * 1e-3) / 1e12 / tflops_peak, 4),
+                     "traffic": None, "kernel": "fwd_kernel<64, fp16, causal>",
+                     "peak_source": f"{peak_src} bf16 burst (fp16 dense rate equals bf16)"},
+        "gpu_launches": K * (2 + (1 if splits > 1 else 0)),
+        "clocks": clk.summary(),
+    }
+    if not args.no_e2e:
+        res["e2e"] = e2e_prefill(fa, q, k, v, dev, stream, flops, world)
+    return res
+
+
+def e2e_prefill(fa, q, k, v, dev, stream, flops, world, steps=5):
+    """Prefill TFLOPS through the public call with pinned host buffers: the H2D copy
+    of q, k, v, the kernel and the D2H copy of O are all inside the timed region."""
+    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    hout = torch.empty_like(hq).pin_memory()
+    dq_, dk_, dv_ = torch.empty_like(hq, device=dev), torch.empty_like(hk, device=dev), \
+        torch.empty_like(hv, device=dev)
+    dout = torch.empty_like(dq_)
+    for _ in range(2):
+        dq_.copy_(hq, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        dq_.copy_(hq, non_blocking=True)
+        dk_.copy_(hk, non_blocking=True)
+        dv_.copy_(hv, non_blocking=True)
+        fa.fa_fwd(dq_, dk_, dv_, out=dout, causal=True, return_lse=False, stream=stream)
+        hout.copy_(dout, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    ms = max_over_ranks(ms, world)
+    h2d = 3 * hq.numel() * hq.element_size()
+    d2h = hout.numel() * hout.element_size()
+    return {"value": round(flops / (ms * 1e-3) / 1e12 * world, 2), "unit": "TFLOPS",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "what": "prefill via fa_fwd with pinned host inputs/outputs copied every step"}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_prefill_sample(heads: int, threads: int):
+    """Time the fp64 oracle on `heads` full (b=0, h) problems of the prefill workload."""
+    import oracle
+    c = PREFILL
+    q, k, v = synth.dense(1, c["S"], c["S"], heads, heads, c["d"], synth.DTYPES[c["dtype"]],
+                          seed=1003)
+    t0 = time.perf_counter()
+    oracle.attention_dense(q, k, v, causal=True, threads=threads)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * c["d"] * heads * causal_pairs(c["S"], c["S"])
+    return flops / dt / 1e12, dt
+
+
+def cpu_baseline(args):
+    heads = max(1, min(32, os.cpu_count() or 1))       # one OpenMP thread per head
+    tf, dt = oracle_prefill_sample(heads, heads)
+    return {"value": round(tf, 6), "unit": "TFLOPS", "cores": heads, "kind": "oracle",
+            "sample": f"prefill workload, batch 0, {heads} of 32 heads, full S=4096 causal "
+                      f"(fp64 C oracle, OpenMP over heads), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 CPU oracle on bounded samples of the prefill workload."""
+    heads = max(1, min(8, os.cpu_count() or 1))        # one OpenMP thread per head
+    cores = heads
+    times = []
+    for i in range(args.warmup + args.steps):
+        tf, dt = oracle_prefill_sample(heads, heads)
+        if i >= args.warmup:
+            times.append((tf, dt))
+    tf = statistics.median(t for t, _ in times)
+    ms = statistics.median(d for _, d in times) * 1e3
+    return {"metric": METRIC, "impl": "reference", "value": round(tf, 6), "unit": "TFLOPS",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": "causal prefill B=4 S=4096 H=32 d=64 (bounded sample: "
+                                   f"batch 0, {heads} heads per step)"},
+            "cpu_baseline": {"value": round(tf, 6), "unit": "TFLOPS", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{heads} heads x full S=4096 causal per step"},
+            "e2e": {"value": round(tf, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--num-splits", type=int, default=16)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps(run_reference(args, rank, world)), flush=True)
+            return
+        res = run_ours(args, rank, world, local)
+        if rank == 0:
+            if not args.no_cpu_baseline and world == 1:
+                res["cpu_baseline"] = cpu_baseline(args)
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

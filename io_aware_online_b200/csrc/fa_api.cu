@@ -148,6 +148,11 @@ int check_common(int dtype, int head_dim, int H, int Hkv, int wl, int wr, float 
 void fill_score_params(float scale, float softcap, float* scale_log2, float* softcap_log2,
                        float* tanh_k) {
   const float log2e = 1.4426950408889634f;
+  // softmax_scale = 0 makes every score 0.  The kernels fold the scale into the
+  // exponent and rely on it being positive (-inf * scale must stay -inf), so 0 is
+  // evaluated as 1e-30: |score| * 1e-30 stays below 2^-24 for any fp16/bf16
+  // input, so every exp2 is exactly 1.0f and the LSE moves by < 1e-18.
+  if (scale == 0.f) scale = 1e-30f;
   *scale_log2 = scale * log2e;
   *softcap_log2 = softcap > 0.f ? softcap * log2e : 0.f;
   *tanh_k = softcap > 0.f ? 2.f * log2e * scale / softcap : 0.f;

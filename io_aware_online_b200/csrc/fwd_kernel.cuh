@@ -7,11 +7,14 @@
 // "FlashAttention common interfaces" sections 3.1/3.2; the causal mask is
 // aligned bottom-right (changelog post, v2.1).
 //
-// CTA = two 128-row query tiles of one (sequence, head); 320 threads:
+// CTA = two 128-row query tiles of one (sequence, head); 384 threads:
 //   warps 0-3  softmax warpgroup of tile 0 (thread r owns query row r = TMEM lane r)
 //   warps 4-7  softmax warpgroup of tile 1
 //   warp  8    TMA producer: Q once, then K_j / V_j blocks into a ring of stages
 //   warp  9    tensor-memory allocator and single-thread tcgen05.mma issuer
+//   warps 10-11 idle (they complete the third warpgroup for the register re-split:
+//              the softmax warpgroups hold a 128-float score row per thread and
+//              take 208 registers; the third warpgroup keeps 80)
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   S_t = Q_t K_j^T   at columns [128 t, 128 t + 128)        (t = 0, 1)
 //   P_t (16-bit)      aliases the first 64 columns of S_t (two values per column)
@@ -37,7 +40,10 @@ namespace fa {
 
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per K/V block
-constexpr int kFwdThreads = 320;
+constexpr int kFwdThreads = 384;
+// 2*128*208 + 128*80 = 63488 <= 384*168 = 64512 (the registers the CTA launches with)
+constexpr uint32_t kSoftmaxRegs = 208;
+constexpr uint32_t kOtherRegs = 80;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
@@ -157,8 +163,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const WaitCtx w{abort_flag, p.status, p.timeout_ns};
   const bool varlen = p.cu_q != nullptr;
   const int b_coord = varlen ? 0 : b;
-
-  if (warp == 8) {
+  if (warp >= 8) {
+   regs_dec<kOtherRegs>();
+   if (warp == 8) {
     // ======================================================== TMA producer
     if (lane == 0 && n_blk > 0) {
       tma_prefetch_map(&tmQ);
@@ -199,7 +206,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+   } else if (warp == 9) {
     // ======================================================== MMA issuer
     if (lane == 0 && n_blk > 0) {
       constexpr uint32_t idesc_qk = f16_idesc(BF16, kBM, kBN, false, false);
@@ -272,7 +279,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       wait_drain(drain, 0, p.timeout_ns);
     }
     __syncwarp();
+   }
   } else {
+    regs_inc<kSoftmaxRegs>();
     // ======================================================== softmax warpgroups
     const int t = warp / 4;
     const int r = threadIdx.x % kBM;
@@ -287,7 +296,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const float slope2 = ALIBI ? p.alibi[h] * kLog2e : 0.f;
     const float ipo = static_cast<float>(i + off);
     float m_use = -INFINITY;  // running max, base-2 units
-    float l = 0.f;            // running sum of exp2(x - m_use)
+    float l = 0.f;            // running sum of exp2(x - m_use): gives the LSE
+    float lr = 0.f;           // the same sum over P rounded to 16 bits: normalises O
     bool ok = true;
 
     for (int it = 0; it < n_blk; ++it) {
@@ -305,14 +315,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int c = 0; c < kBN / 32; ++c) tmem_ld_wait(s + c * 32);
 
       const bool masked = (kb < lo_rb) || (kb + kBN - 1 > hi_ra);
-      const bool plain = !SOFTCAP && !ALIBI && !masked;
+      const int lo_c = lo_i - kb, hi_c = hi_i - kb;  // allowed columns: lo_c <= c <= hi_c
       float m_blk = -INFINITY;
-      if (plain) {
-        // scale folded into the exponent below (softmax_scale >= 0 keeps the order)
+      float factor;  // exponent = s * factor - m
+      if constexpr (!SOFTCAP && !ALIBI) {
+        // raw-score domain: mask, take the max, fold the scale into the exponent
+        // (softmax_scale > 0 here: the host maps 0 to a tiny positive scale)
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            s[c] = (c >= lo_c && c <= hi_c) ? s[c] : __float_as_uint(-INFINITY);
+        }
 #pragma unroll
         for (int c = 0; c < kBN; ++c) m_blk = fmaxf(m_blk, __uint_as_float(s[c]));
         m_blk *= p.scale_log2;
+        factor = p.scale_log2;
       } else {
+        const float base = ipo - static_cast<float>(kb);  // ALiBi distance of column c: |base - c|
 #pragma unroll
         for (int c = 0; c < kBN; ++c) {
           float x = __uint_as_float(s[c]);
@@ -324,16 +343,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           } else {
             x *= p.scale_log2;
           }
-          if constexpr (ALIBI) {
-            x = fmaf(-slope2, fabsf(ipo - static_cast<float>(kb + c)), x);
-          }
-          if (masked) {
-            const int kk = kb + c;
-            x = (kk >= lo_i && kk <= hi_i) ? x : -INFINITY;
-          }
+          if constexpr (ALIBI) x = fmaf(-slope2, fabsf(base - static_cast<float>(c)), x);
+          if (masked) x = (c >= lo_c && c <= hi_c) ? x : -INFINITY;
           s[c] = __float_as_uint(x);
           m_blk = fmaxf(m_blk, x);
         }
+        factor = 1.f;
       }
       // ---- online softmax bookkeeping (lazy rescale)
       const float m_new = fmaxf(m_use, m_blk);
@@ -346,7 +361,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         alpha = ex2(m_use - m_new);
         m_use = m_new;
         l *= alpha;
+        lr *= alpha;
       }
+      // ---- probabilities -> 16-bit P in tensor memory (aliasing S)
+      const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+      float2 lsum = make_float2(0.f, 0.f);
+      float2 lrnd = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int q4 = 0; q4 < kBN / 32; ++q4) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[q4 * 32 + 2 * e]), factor, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(s[q4 * 32 + 2 * e + 1]), factor, neg_m));
+          pk[e] = pack2<BF16>(p0, p1);
+          lsum = add2(lsum, make_float2(p0, p1));
+          // bf16 P is rounded by up to 2^-9: sum the rounded values the PV product
+          // uses, so that O / lr is an exact convex combination of V rows
+          if constexpr (BF16) lrnd = add2(lrnd, unpack2<true>(pk[e]));
+        }
+        tmem_st16(tS + q4 * 16, pk);
+      }
+      l += lsum.x + lsum.y;
+      lr += BF16 ? (lrnd.x + lrnd.y) : (lsum.x + lsum.y);
+      // O_t rescale (after the score row is dead: lower register peak); it only
+      // has to land before P_t is released to the MMA warp
       if (__any_sync(0xffffffffu, need)) {
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
@@ -358,23 +397,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tmem_st32(tO + c * 32, o);
         }
       }
-      // ---- probabilities -> 16-bit P in tensor memory (aliasing S)
-      const float factor = plain ? p.scale_log2 : 1.f;
-      const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
-      float lsum = 0.f;
-#pragma unroll
-      for (int q4 = 0; q4 < kBN / 32; ++q4) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(fmaf(__uint_as_float(s[q4 * 32 + 2 * e]), factor, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(s[q4 * 32 + 2 * e + 1]), factor, neg_m));
-          lsum += p0 + p1;
-          pk[e] = pack2<BF16>(p0, p1);
-        }
-        tmem_st16(tS + q4 * 16, pk);
-      }
-      l += lsum;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full + t);
@@ -386,7 +408,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (ok) {
       tc_fence_after();
       const bool row_ok = i < Sq_b;
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv = (lr > 0.f) ? 1.f / lr : 0.f;
       uint8_t* orow = nullptr;
       if (row_ok) {
         const int64_t ro = varlen ? static_cast<int64_t>(q0 + i) * p.o_ss

@@ -70,7 +70,8 @@ struct WaitCtx {
 
 // Wait until phase `parity` of `bar` has completed.  Returns false (and leaves the
 // CTA marked aborted) if the limit ran out or another role aborted first.
-static __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+// (inlined: a real call inside a setmaxnreg region defeats register allocation)
+__device__ __forceinline__ bool wait_slow(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -250,6 +251,16 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Warpgroup-wide register re-split (all four warps of a warpgroup execute it).
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ----------------------------------------------------------------- math
 // Hardware base-2 exponential (MUFU), flushing subnormals; exp2(-inf) = +0.
 __device__ __forceinline__ float ex2(float x) {
@@ -262,6 +273,23 @@ __device__ __forceinline__ float rcp(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed fp32 pair arithmetic (one instruction for two lanes of work on sm_100).
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
+  return *reinterpret_cast<float2*>(&r);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
+        "l"(*reinterpret_cast<uint64_t*>(&c)));
+  return *reinterpret_cast<float2*>(&r);
 }
 
 // Two fp32 values rounded to the 16-bit input type, lower index in the low half.
