@@ -190,6 +190,8 @@ def run_ours(args, rank, world, local):
     qd_, kd_, vd_ = q.to(dev), k.to(dev), v.to(dev)
     out_p = torch.empty_like(qd_)
     lse_p = torch.empty((PREFILL["B"], PREFILL["H"], PREFILL["S"]), dtype=torch.float32, device=dev)
+    if args.only == "prefill":        # keep the decode pool tiny when it is not timed
+        DECODE.update(B=2, lo=1024, hi=1024)
     dq, kp, vp, bt, cs, lens = make_decode(rank, dev)
     dq_d, bt_d, cs_d = dq.to(dev), bt.to(dev), cs.to(dev)
     splits = args.num_splits
@@ -202,12 +204,18 @@ def run_ours(args, rank, world, local):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
     stream = torch.cuda.current_stream(dev)
 
+    do_pre = args.only in ("all", "prefill")
+    do_dec = args.only in ("all", "decode")
+
     def prefill():
-        fa.fa_fwd(qd_, kd_, vd_, out=out_p, lse=lse_p, causal=True, stream=stream)
+        if do_pre:
+            fa.fa_fwd(qd_, kd_, vd_, out=out_p, lse=lse_p, causal=True, stream=stream)
 
     def decode():
-        fa.fa_fwd_kvcache(dq_d, kp, vp, cache_seqlens=cs_d, block_table=bt_d, causal=True,
-                          num_splits=splits, out=out_d, lse=lse_d, workspace=ws, stream=stream)
+        if do_dec:
+            fa.fa_fwd_kvcache(dq_d, kp, vp, cache_seqlens=cs_d, block_table=bt_d, causal=True,
+                              num_splits=splits, out=out_d, lse=lse_d, workspace=ws,
+                              stream=stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -230,6 +238,8 @@ def run_ours(args, rank, world, local):
     barrier(world)
     t_pre = sum(e[0].elapsed_time(e[1]) for e in ev) / K      # ms per launch
     t_dec = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    t_pre = max(t_pre, 1e-9)
+    t_dec = max(t_dec, 1e-9)
     t_step = t_pre + t_dec
     t_pre_max = max_over_ranks(t_pre, world)
     t_dec_max = max_over_ranks(t_dec, world)
@@ -254,8 +264,9 @@ def run_ours(args, rank, world, local):
         "dtype": "fp16 (prefill), bf16 (decode); fp32 accumulate",
         "data": "synthetic (seeded N(0,1))",
         "config": {
-            "workload": "causal prefill B=4 S=4096 H=32 d=64 fp16 + paged split-KV decode "
-                        "B=64 H=32 Hkv=8 d=128 bf16 cache U{1K..32K} page 256",
+            "workload": (f"causal prefill B={PREFILL['B']} S={PREFILL['S']} H={PREFILL['H']} "
+                         f"d={PREFILL['d']} {PREFILL['dtype']} + paged split-KV decode "
+                         f"B={DECODE['B']} H=32 Hkv=8 d=128 bf16 cache U{{1K..32K}} page 256"),
             "prefill": dict(PREFILL, ms=round(t_pre_max, 4), flop=flops),
             "decode": dict(DECODE, num_splits=splits, sum_cache_tokens=int(sum(lens)),
                            ms=round(t_dec_max, 4), bytes=dbytes),
@@ -272,9 +283,10 @@ def run_ours(args, rank, world, local):
         "roofline": {"bound": "tensor", "achieved": round(flops / (t_pre * 1e-3) / 1e12, 2),
                      "peak": tflops_peak, "unit": "TFLOP/s",
                      "frac": round(flops / (t_pre * 1e-3) / 1e12 / tflops_peak, 4),
-                     "traffic": None, "kernel": "fwd_kernel<64, fp16, causal>",
+                     "traffic": None,
+                     "kernel": f"fwd_kernel<{PREFILL['d']}, {PREFILL['dtype']}, causal>",
                      "peak_source": f"{peak_src} bf16 burst (fp16 dense rate equals bf16)"},
-        "gpu_launches": K * (2 + (1 if splits > 1 else 0)),
+        "gpu_launches": K * ((1 if do_pre else 0) + ((2 if splits > 1 else 1) if do_dec else 0)),
         "clocks": clk.summary(),
     }
     if not args.no_e2e:
@@ -367,7 +379,15 @@ def main():
     ap.add_argument("--num-splits", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="time one part of the step (profiling / sweeps)")
+    ap.add_argument("--prefill-seq", type=int, default=PREFILL["S"])
+    ap.add_argument("--prefill-d", type=int, default=PREFILL["d"])
+    ap.add_argument("--prefill-dtype", choices=["fp16", "bf16"], default=PREFILL["dtype"])
+    ap.add_argument("--decode-batch", type=int, default=DECODE["B"])
     args = ap.parse_args()
+    PREFILL.update(S=args.prefill_seq, d=args.prefill_d, dtype=args.prefill_dtype)
+    DECODE.update(B=args.decode_batch)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     rank, world, local = dist_setup(args.gpus)

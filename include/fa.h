@@ -111,8 +111,9 @@ FA_API int fa_kvcache_num_splits(int batch, int seqlen_q, int num_heads, int num
 
 /*
  * fa_kvcache_workspace_size -- bytes of device scratch fa_fwd_kvcache needs:
- * splits * batch * seqlen_q * num_heads * (head_dim + 1) * 4 when the resolved split
- * count is above 1, else 0.  Same arguments as fa_kvcache_num_splits.
+ * 256 (a work-item counter the call resets) plus, when the resolved split count is
+ * above 1, splits * batch * seqlen_q * num_heads * (head_dim + 1) * 4 for the fp32
+ * split partials.  Same arguments as fa_kvcache_num_splits.
  */
 FA_API size_t fa_kvcache_workspace_size(int batch, int seqlen_q, int num_heads, int num_heads_k,
                                  int head_dim, int max_seqlen_k, int page_size,
@@ -140,9 +141,11 @@ FA_API size_t fa_kvcache_workspace_size(int batch, int seqlen_q, int num_heads, 
  *   ranges of ceil(pages / num_splits) pages, each computed by its own CTAs, and a
  *   second kernel combines them (fa_combine's arithmetic).  The result does not
  *   depend on num_splits beyond rounding.
- * workspace: device scratch of at least fa_kvcache_workspace_size(...) bytes
- *   (may be NULL when that is 0); it holds the fp32 split partials between the
- *   two kernels of one call, so calls that share it must be stream-ordered.
+ * workspace: device scratch of at least fa_kvcache_workspace_size(...) bytes,
+ *   16-byte aligned, required.  It holds the split kernel's work-item counter
+ *   (zeroed by the call with an asynchronous memset on `stream`) and the fp32
+ *   split partials between the two kernels of one call, so calls that share a
+ *   workspace must be stream-ordered.
  * Limits: num_heads / num_heads_k * seqlen_q <= 16 rows per KV head.
  */
 FA_API int fa_fwd_kvcache(const void *q, const void *k_cache, const void *v_cache, void *out, float *lse,

@@ -208,7 +208,7 @@ def fa_fwd_kvcache(q, k_cache, v_cache, *, cache_seqlens=None, block_table=None,
         sk_max, Hkv = k_cache.shape[1], k_cache.shape[2]
         max_k = sk_max
     need = fa_kvcache_workspace_size(B, sq, H, Hkv, d, max_k, page, num_splits)
-    if workspace is None and need > 0:
+    if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     if out is None:

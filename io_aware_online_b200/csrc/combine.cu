@@ -53,19 +53,67 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Combi
   __syncwarp();
 
   const int64_t out_row = row * p.D;
-  for (int dd = lane; dd < p.D; dd += 32) {
-    float acc = 0.f;
-    const float* col = orow + dd * p.op_s[3];
-    for (int sp = 0; sp < p.splits; ++sp) {
-      const float wv = wts[warp][sp];
-      if (wv != 0.f) acc = fmaf(wv, col[sp * p.op_s[4]], acc);
+  if (p.op_s[3] == 1 && (p.op_s[4] % 4) == 0 && ((reinterpret_cast<uintptr_t>(orow) & 15) == 0)) {
+    // head dim contiguous: each lane owns 4 consecutive columns (one 16-byte load
+    // per split), and the split loop is unrolled so that loads overlap
+    for (int d0 = lane * 4; d0 < p.D; d0 += 128) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      int sp = 0;
+      for (; sp + 4 <= p.splits; sp += 4) {
+        float4 v[4];
+        float wv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          wv[u] = wts[warp][sp + u];
+          v[u] = wv[u] != 0.f ? *reinterpret_cast<const float4*>(orow + (sp + u) * p.op_s[4] + d0)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          acc.x = fmaf(wv[u], v[u].x, acc.x);
+          acc.y = fmaf(wv[u], v[u].y, acc.y);
+          acc.z = fmaf(wv[u], v[u].z, acc.z);
+          acc.w = fmaf(wv[u], v[u].w, acc.w);
+        }
+      }
+      for (; sp < p.splits; ++sp) {
+        const float wv = wts[warp][sp];
+        if (wv == 0.f) continue;
+        const float4 v = *reinterpret_cast<const float4*>(orow + sp * p.op_s[4] + d0);
+        acc.x = fmaf(wv, v.x, acc.x);
+        acc.y = fmaf(wv, v.y, acc.y);
+        acc.z = fmaf(wv, v.z, acc.z);
+        acc.w = fmaf(wv, v.w, acc.w);
+      }
+      // head_dim is a multiple of 4 (checked by the host), so all four columns exist
+      if constexpr (OUT_DT == 0) {
+        __half* o = static_cast<__half*>(p.out) + out_row + d0;
+        o[0] = __float2half_rn(acc.x); o[1] = __float2half_rn(acc.y);
+        o[2] = __float2half_rn(acc.z); o[3] = __float2half_rn(acc.w);
+      } else if constexpr (OUT_DT == 1) {
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + out_row + d0;
+        o[0] = __float2bfloat16_rn(acc.x); o[1] = __float2bfloat16_rn(acc.y);
+        o[2] = __float2bfloat16_rn(acc.z); o[3] = __float2bfloat16_rn(acc.w);
+      } else {
+        float* o = static_cast<float*>(p.out) + out_row + d0;
+        o[0] = acc.x; o[1] = acc.y; o[2] = acc.z; o[3] = acc.w;
+      }
     }
-    if constexpr (OUT_DT == 0)
-      static_cast<__half*>(p.out)[out_row + dd] = __float2half_rn(acc);
-    else if constexpr (OUT_DT == 1)
-      static_cast<__nv_bfloat16*>(p.out)[out_row + dd] = __float2bfloat16_rn(acc);
-    else
-      static_cast<float*>(p.out)[out_row + dd] = acc;
+  } else {
+    for (int dd = lane; dd < p.D; dd += 32) {
+      float acc = 0.f;
+      const float* col = orow + dd * p.op_s[3];
+      for (int sp = 0; sp < p.splits; ++sp) {
+        const float wv = wts[warp][sp];
+        if (wv != 0.f) acc = fmaf(wv, col[sp * p.op_s[4]], acc);
+      }
+      if constexpr (OUT_DT == 0)
+        static_cast<__half*>(p.out)[out_row + dd] = __float2half_rn(acc);
+      else if constexpr (OUT_DT == 1)
+        static_cast<__nv_bfloat16*>(p.out)[out_row + dd] = __float2bfloat16_rn(acc);
+      else
+        static_cast<float*>(p.out)[out_row + dd] = acc;
+    }
   }
   if (lane == 0 && p.lse != nullptr)
     p.lse[(static_cast<int64_t>(b) * p.H + h) * p.S + s] = lse;

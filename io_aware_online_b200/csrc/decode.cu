@@ -1,4 +1,6 @@
 // decode.cu -- instantiation and launch of the split-KV decode kernel.
+#include <algorithm>
+
 #include "decode_kernel.cuh"
 
 namespace fa {
@@ -10,9 +12,15 @@ static cudaError_t launch_decode_inst(const CUtensorMap& tk, const CUtensorMap& 
   constexpr int smem = DecCfg<D, RMAX>::kSmemAlloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(p.num_splits), static_cast<unsigned>(p.Hkv),
-                  static_cast<unsigned>(p.B));
-  kern<<<grid, kDecThreads, smem, stream>>>(tk, tv, p);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  // persistent grid: as many CTAs as fit at once, each walking the item list
+  const long items = static_cast<long>(p.B) * p.Hkv * p.num_splits;
+  const long per_sm = (RMAX <= 4) ? 3 : 1;
+  const long ctas = std::min(items, per_sm * std::max(1, p.sm_count));
+  if (ctas <= 0) return cudaSuccess;
+  kern<<<static_cast<unsigned>(ctas), kDecThreads, smem, stream>>>(tk, tv, p);
   return cudaGetLastError();
 }
 

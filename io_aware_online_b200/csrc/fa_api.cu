@@ -164,9 +164,10 @@ int resolve_splits(int batch, int Sq, int H, int Hkv, int d, int max_seqlen_k, i
   if (batch < 0 || Hkv <= 0 || max_seqlen_k < 0 || unit <= 0 || num_splits < 0) return -1;
   const int units = std::max(1, (max_seqlen_k + unit - 1) / unit);
   if (num_splits > 0) return std::min(num_splits, units);
-  // heuristic: enough CTAs for about four waves of two CTAs per SM
+  // heuristic: about eight work items per resident decode CTA (three per SM), so the
+  // persistent CTAs finish together despite unequal sequence lengths
   const long ctas = std::max(1L, static_cast<long>(batch) * Hkv);
-  const long want = 8L * sm_count_or_default();
+  const long want = 24L * sm_count_or_default();
   long s = (want + ctas - 1) / ctas;
   s = std::min<long>(s, std::min(units, 64));
   return static_cast<int>(std::max(1L, s));
@@ -305,12 +306,19 @@ int fa_kvcache_num_splits(int batch, int seqlen_q, int num_heads, int num_heads_
                         num_splits);
 }
 
+// Workspace layout: a 256-byte header (word 0: the decode kernel's work-item counter,
+// zeroed at every call) followed, when the split count is above 1, by the fp32
+// partial outputs [splits, B, Sq, H, D] and partial LSEs [splits, B, Sq, H].
+static constexpr size_t kWsHeader = 256;
+
 size_t fa_kvcache_workspace_size(int batch, int seqlen_q, int num_heads, int num_heads_k,
                                  int head_dim, int max_seqlen_k, int page_size, int num_splits) {
   const int s = fa_kvcache_num_splits(batch, seqlen_q, num_heads, num_heads_k, head_dim,
                                       max_seqlen_k, page_size, num_splits);
-  if (s <= 1 || batch <= 0 || seqlen_q <= 0 || num_heads <= 0 || head_dim <= 0) return 0;
-  return static_cast<size_t>(s) * batch * seqlen_q * num_heads * (head_dim + 1) * sizeof(float);
+  if (s <= 0 || batch <= 0 || seqlen_q <= 0 || num_heads <= 0 || head_dim <= 0) return kWsHeader;
+  if (s == 1) return kWsHeader;
+  return kWsHeader +
+         static_cast<size_t>(s) * batch * seqlen_q * num_heads * (head_dim + 1) * sizeof(float);
 }
 
 int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void* out, float* lse,
@@ -358,12 +366,13 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
   const int splits = resolve_splits(batch, seqlen_q, H, Hkv, d, max_k, unit, num_splits);
   const size_t need = fa_kvcache_workspace_size(batch, seqlen_q, H, Hkv, d, max_k,
                                                 paged ? page_size : 0, num_splits);
-  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
     return fail(FA_ERR_WORKSPACE, "fa_fwd_kvcache: needs %zu bytes of 16-byte aligned workspace (got %zu)",
                 need, workspace_bytes);
   if ((rc = get_encoder()) != FA_OK) return rc;
   unsigned int* status = nullptr;
-  if ((rc = device_state(nullptr, &status, nullptr)) != FA_OK) return rc;
+  int sms = 0;
+  if ((rc = device_state(nullptr, &status, &sms)) != FA_OK) return rc;
 
   CUtensorMap tk, tv;
   const uint32_t box[4] = {64, 1, 64, 1};
@@ -388,10 +397,11 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
   p.q = q;
   p.out = out;
   p.lse = lse;
-  p.ws_o = static_cast<float*>(workspace);
-  p.ws_lse = splits > 1 ? static_cast<float*>(workspace) +
-                              static_cast<size_t>(splits) * batch * seqlen_q * H * d
+  float* ws_parts = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWsHeader);
+  p.ws_o = splits > 1 ? ws_parts : nullptr;
+  p.ws_lse = splits > 1 ? ws_parts + static_cast<size_t>(splits) * batch * seqlen_q * H * d
                         : nullptr;
+  p.item_counter = static_cast<unsigned int*>(workspace);
   p.block_table = block_table;
   p.cache_seqlens = cache_seqlens;
   p.B = batch;
@@ -414,8 +424,11 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
   p.wr = window_right;
   p.status = status;
   p.timeout_ns = timeout_ns();
+  p.sm_count = sms;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = fa::launch_decode(tk, tv, p, dtype == FA_BF16, d, s);
+  cudaError_t e = cudaMemsetAsync(p.item_counter, 0, sizeof(unsigned int), s);
+  if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache counter reset");
+  e = fa::launch_decode(tk, tv, p, dtype == FA_BF16, d, s);
   if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache split kernel launch");
   if (splits > 1) {
     fa::CombineParams c{};

@@ -50,6 +50,8 @@ struct DecodeParams {
   int causal, wl, wr;
   unsigned int* status;
   uint64_t timeout_ns;
+  int sm_count;                    // persistent grid: CTAs per SM x sm_count (capped at items)
+  unsigned int* item_counter;      // workspace word, zero at launch: next work item to claim
 };
 
 cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,

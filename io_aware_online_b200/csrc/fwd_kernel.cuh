@@ -14,7 +14,7 @@
 //   warp  9    tensor-memory allocator and single-thread tcgen05.mma issuer
 //   warps 10-11 idle (they complete the third warpgroup for the register re-split:
 //              the softmax warpgroups hold a 128-float score row per thread and
-//              take 208 registers; the third warpgroup keeps 80)
+//              take 200 registers; the third warpgroup keeps 104)
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   S_t = Q_t K_j^T   at columns [128 t, 128 t + 128)        (t = 0, 1)
 //   P_t (16-bit)      aliases the first 64 columns of S_t (two values per column)
@@ -41,9 +41,9 @@ namespace fa {
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per K/V block
 constexpr int kFwdThreads = 384;
-// 2*128*208 + 128*80 = 63488 <= 384*168 = 64512 (the registers the CTA launches with)
-constexpr uint32_t kSoftmaxRegs = 208;
-constexpr uint32_t kOtherRegs = 80;
+// 2*128*200 + 128*104 = 64512 = 384*168 (the registers the CTA launches with)
+constexpr uint32_t kSoftmaxRegs = 200;
+constexpr uint32_t kOtherRegs = 104;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
@@ -59,13 +59,19 @@ struct FwdCfg {
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
-  // o_final[2], drain
-  static constexpr int kNumBars = 1 + 4 * kStages + 7;
+  // o_final[2], drain, s_free[2], pv_done[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 11;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // room to align the base to 1 KiB
   static constexpr int kTmemCols = 512;
-  static constexpr int kOCol = 256;
+  // D = 64: P has its own columns (S 2x128, P 2x64, O 2x64 = 512), so the next
+  // S can be computed while the softmax still works on the current one.
+  // D = 128: S 2x128 + O 2x128 fill the 512 columns and P aliases S.
+  static constexpr bool kSepP = (D == 64);
+  static constexpr int kPCol = kSepP ? 256 : 0;
+  static constexpr int kPStride = kSepP ? 64 : 128;
+  static constexpr int kOCol = kSepP ? 384 : 256;
 };
 
 // Wait that ignores the abort flag (used to drain this CTA's own in-flight work).
@@ -77,7 +83,33 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint6
   return true;
 }
 
-template <int D, bool BF16, bool SOFTCAP, bool ALIBI>
+// EMU: of every 8 pairs of probabilities, EMU are evaluated by exp2_fma2 on the
+// FMA pipe and the rest by the MUFU unit (balances the two at small head dims).
+// S_t = Q_t K^T into tensor memory: K-major A (Q tile) and B (K block); a step of
+// 16 along the head dim is 32 bytes inside a 128-byte swizzle atom, the next atom
+// lies 16 KiB further.
+template <int D>
+__device__ __forceinline__ void fwd_issue_qk(uint32_t d_tmem, uint64_t a0, uint64_t b0,
+                                             uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
+    mma_ss(d_tmem, desc_advance(a0, o), desc_advance(b0, o), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O_t (+)= P_t V: A = P from tensor memory (8 columns hold 16 keys), B = V block,
+// MN-major (16 keys = 16 rows = 2 KiB; head-dim atoms 16 KiB apart).
+template <int D>
+__device__ __forceinline__ void fwd_issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
+                                             uint32_t idesc, bool acc) {
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk)
+    mma_ts(d_tmem, a_tmem + kk * 8, desc_advance(b0, kk * 2048), idesc,
+           (acc || kk > 0) ? 1u : 0u);
+}
+
+template <int D, bool BF16, bool SOFTCAP, bool ALIBI, int EMU>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -132,6 +164,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* p_full = bars + 3 + 4 * ST;
   uint64_t* o_final = bars + 5 + 4 * ST;
   uint64_t* drain = bars + 7 + 4 * ST;
+  uint64_t* s_free = bars + 8 + 4 * ST;   // softmax has S_t in registers (separate-P layout)
+  uint64_t* pv_done = bars + 10 + 4 * ST; // PV_t finished: P_t may be rewritten, O_t rescaled
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -147,6 +181,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(s_full + t, 1);
       mbar_init(p_full + t, kBM);
       mbar_init(o_final + t, 1);
+      mbar_init(s_free + t, kBM);
+      mbar_init(pv_done + t, 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -211,32 +247,68 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (lane == 0 && n_blk > 0) {
       constexpr uint32_t idesc_qk = f16_idesc(BF16, kBM, kBN, false, false);
       constexpr uint32_t idesc_pv = f16_idesc(BF16, kBM, D, false, true);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      // S_t = Q_t K^T: K-major A and B; step 16 of the head dim = 32 bytes inside a
-      // 128-byte swizzle atom, the next atom 16 KiB further.
-      auto qk = [&](int t, int s) {
-        const uint32_t d_tmem = tbase + t * kBM;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t o = (kk / 4) * Cfg::kChunkBytes + (kk % 4) * 32;
-          mma_ss(d_tmem, sw128_desc(aQ + t * Cfg::kTileBytes + o, 16, 1024),
-                 sw128_desc(aK + s * Cfg::kTileBytes + o, 16, 1024), idesc_qk, kk > 0);
-        }
-      };
-      // O_t += P_t V: A = P from tensor memory (8 columns per 16 keys), B = V
-      // MN-major (keys advance 16 rows = 2 KiB, head-dim atoms 16 KiB apart).
-      auto pv = [&](int t, int s, bool acc) {
-        const uint32_t d_tmem = tbase + Cfg::kOCol + t * D;
-        const uint32_t a_tmem = tbase + t * kBM;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts(d_tmem, a_tmem + kk * 8,
-                 sw128_desc(aV + s * Cfg::kTileBytes + kk * 2048, Cfg::kChunkBytes, 1024),
-                 idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        }
-      };
+      // Descriptor bases computed once; every MMA below forms its operand
+      // descriptors with one add on the low word (the issuing thread is on the
+      // critical path of the pipeline, so its per-instruction work stays small).
+      const uint64_t dQ = sw128_desc(smem_u32(sQ), 16, 1024);               // K-major
+      const uint64_t dK = sw128_desc(smem_u32(sK), 16, 1024);               // K-major
+      const uint64_t dV = sw128_desc(smem_u32(sV), Cfg::kChunkBytes, 1024); // MN-major
+      const uint32_t tS0 = tbase, tS1 = tbase + kBM;
+      const uint32_t tP0 = tbase + Cfg::kPCol, tP1 = tbase + Cfg::kPCol + Cfg::kPStride;
+      const uint32_t tO0 = tbase + Cfg::kOCol, tO1 = tbase + Cfg::kOCol + D;
+      const uint64_t dQ0 = dQ, dQ1 = desc_advance(dQ, Cfg::kTileBytes);
+#define FA_QK(T, S)                                                                         \
+  fwd_issue_qk<D>(T ? tS1 : tS0, T ? dQ1 : dQ0, desc_advance(dK, (S) * Cfg::kTileBytes),   \
+                  idesc_qk)
+#define FA_PV(T, S, ACC)                                                                    \
+  fwd_issue_pv<D>(T ? tO1 : tO0, T ? tP1 : tP0, desc_advance(dV, (S) * Cfg::kTileBytes),   \
+                  idesc_pv, ACC)
+#define qk(T, S) FA_QK(T, S)
+#define pv(T, S, ACC) FA_PV(T, S, ACC)
       bool ok = wait_bounded(q_full, 0, w) && wait_bounded(k_full, 0, w);
-      if (ok) {
+      if (ok && Cfg::kSepP) {
+        // QK_t(j+1) as soon as softmax t holds S_t(j) in registers; PV_t(j) when P_t(j)
+        // is written.  Each tile's softmax then runs back to back.
+        tc_fence_after();
+        qk(0, 0);
+        tc_commit(s_full + 0);
+        qk(1, 0);
+        tc_commit(s_full + 1);
+        tc_commit(k_empty + 0);
+        for (int it = 0; it < n_blk && ok; ++it) {
+          const int s = it % ST;
+          const uint32_t ph = (it / ST) & 1;
+          const bool more = it + 1 < n_blk;
+          const int s1 = (it + 1) % ST;
+          const uint32_t ph1 = ((it + 1) / ST) & 1;
+          if (more) {
+            if (!(ok = wait_bounded(k_full + s1, ph1, w))) break;
+            if (!(ok = wait_bounded(s_free + 0, it & 1, w))) break;
+            tc_fence_after();
+            qk(0, s1);
+            tc_commit(s_full + 0);
+          }
+          if (!(ok = wait_bounded(v_full + s, ph, w))) break;
+          if (!(ok = wait_bounded(p_full + 0, it & 1, w))) break;
+          tc_fence_after();
+          pv(0, s, it > 0);
+          tc_commit(pv_done + 0);
+          if (!more) tc_commit(o_final + 0);
+          if (more) {
+            if (!(ok = wait_bounded(s_free + 1, it & 1, w))) break;
+            tc_fence_after();
+            qk(1, s1);
+            tc_commit(s_full + 1);
+            tc_commit(k_empty + s1);
+          }
+          if (!(ok = wait_bounded(p_full + 1, it & 1, w))) break;
+          tc_fence_after();
+          pv(1, s, it > 0);
+          tc_commit(pv_done + 1);
+          tc_commit(v_empty + s);
+          if (!more) tc_commit(o_final + 1);
+        }
+      } else if (ok) {
         tc_fence_after();
         qk(0, 0);
         tc_commit(s_full + 0);
@@ -274,6 +346,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
       }
+#undef qk
+#undef pv
+#undef FA_QK
+#undef FA_PV
       // every MMA issued above is complete before tensor memory is released
       tc_commit(drain);
       wait_drain(drain, 0, p.timeout_ns);
@@ -287,6 +363,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int r = threadIdx.x % kBM;
     const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
     const uint32_t tS = tbase + t * kBM + lane_off;
+    const uint32_t tP = tbase + Cfg::kPCol + t * Cfg::kPStride + lane_off;
     const uint32_t tO = tbase + Cfg::kOCol + t * D + lane_off;
     const int i = row0 + t * kBM + r;  // query row within the sequence
     const int ra = row0 + t * kBM;
@@ -313,22 +390,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, s + c * 32);
 #pragma unroll
       for (int c = 0; c < kBN / 32; ++c) tmem_ld_wait(s + c * 32);
+      if constexpr (Cfg::kSepP) {  // S_t may now be overwritten by the next QK
+        tc_fence_before();
+        mbar_arrive(s_free + t);
+      }
 
       const bool masked = (kb < lo_rb) || (kb + kBN - 1 > hi_ra);
       const int lo_c = lo_i - kb, hi_c = hi_i - kb;  // allowed columns: lo_c <= c <= hi_c
-      float m_blk = -INFINITY;
-      float factor;  // exponent = s * factor - m
+      float factor;  // exponent argument = s * factor - m
       if constexpr (!SOFTCAP && !ALIBI) {
-        // raw-score domain: mask, take the max, fold the scale into the exponent
+        // raw-score domain: mask here, fold the scale into the exponent below
         // (softmax_scale > 0 here: the host maps 0 to a tiny positive scale)
         if (masked) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
             s[c] = (c >= lo_c && c <= hi_c) ? s[c] : __float_as_uint(-INFINITY);
         }
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) m_blk = fmaxf(m_blk, __uint_as_float(s[c]));
-        m_blk *= p.scale_log2;
         factor = p.scale_log2;
       } else {
         const float base = ipo - static_cast<float>(kb);  // ALiBi distance of column c: |base - c|
@@ -346,9 +423,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if constexpr (ALIBI) x = fmaf(-slope2, fabsf(base - static_cast<float>(c)), x);
           if (masked) x = (c >= lo_c && c <= hi_c) ? x : -INFINITY;
           s[c] = __float_as_uint(x);
-          m_blk = fmaxf(m_blk, x);
         }
         factor = 1.f;
+      }
+      // ---- row max: four independent chains of three-input max
+      float m_blk;
+      {
+        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kBN; c += 8) {
+          a0 = max3f(a0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+          a1 = max3f(a1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+          a2 = max3f(a2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+          a3 = max3f(a3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+        }
+        m_blk = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * factor;
       }
       // ---- online softmax bookkeeping (lazy rescale)
       const float m_new = fmaxf(m_use, m_blk);
@@ -363,27 +452,50 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         l *= alpha;
         lr *= alpha;
       }
-      // ---- probabilities -> 16-bit P in tensor memory (aliasing S)
+      // ---- probabilities -> 16-bit P in tensor memory
+      if constexpr (Cfg::kSepP) {
+        // P_t(j-1) must have been consumed (and O_t updated) by PV_t(j-1)
+        if (it > 0) {
+          ok = wait_bounded(pv_done + t, (it - 1) & 1, w);
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+      }
       const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
-      float2 lsum = make_float2(0.f, 0.f);
-      float2 lrnd = make_float2(0.f, 0.f);
+      const float2 f2 = make_float2(factor, factor), nm2 = make_float2(neg_m, neg_m);
+      float2 lsum[kBN / 32], lrnd[kBN / 32];
 #pragma unroll
       for (int q4 = 0; q4 < kBN / 32; ++q4) {
         uint32_t pk[16];
+        lsum[q4] = make_float2(0.f, 0.f);
+        lrnd[q4] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(fmaf(__uint_as_float(s[q4 * 32 + 2 * e]), factor, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(s[q4 * 32 + 2 * e + 1]), factor, neg_m));
-          pk[e] = pack2<BF16>(p0, p1);
-          lsum = add2(lsum, make_float2(p0, p1));
+          const float2 arg = fma2(make_float2(__uint_as_float(s[q4 * 32 + 2 * e]),
+                                              __uint_as_float(s[q4 * 32 + 2 * e + 1])),
+                                  f2, nm2);
+          float2 pp;
+          if ((e % 8) < EMU)
+            pp = exp2_fma2(arg);
+          else
+            pp = make_float2(ex2(arg.x), ex2(arg.y));
+          pk[e] = pack2<BF16>(pp.x, pp.y);
+          lsum[q4] = add2(lsum[q4], pp);
           // bf16 P is rounded by up to 2^-9: sum the rounded values the PV product
           // uses, so that O / lr is an exact convex combination of V rows
-          if constexpr (BF16) lrnd = add2(lrnd, unpack2<true>(pk[e]));
+          if constexpr (BF16) lrnd[q4] = add2(lrnd[q4], unpack2<true>(pk[e]));
         }
-        tmem_st16(tS + q4 * 16, pk);
+        tmem_st16(tP + q4 * 16, pk);
       }
-      l += lsum.x + lsum.y;
-      lr += BF16 ? (lrnd.x + lrnd.y) : (lsum.x + lsum.y);
+      {
+        float2 a = add2(add2(lsum[0], lsum[1]), add2(lsum[2], lsum[3]));
+        l += a.x + a.y;
+        if constexpr (BF16) a = add2(add2(lrnd[0], lrnd[1]), add2(lrnd[2], lrnd[3]));
+        lr += a.x + a.y;
+      }
       // O_t rescale (after the score row is dead: lower register peak); it only
       // has to land before P_t is released to the MMA warp
       if (__any_sync(0xffffffffu, need)) {
@@ -408,7 +520,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (ok) {
       tc_fence_after();
       const bool row_ok = i < Sq_b;
-      const float inv = (lr > 0.f) ? 1.f / lr : 0.f;
+      // a row with no allowed key keeps m = -inf (its sum may hold clamped
+      // polynomial exponentials of -inf, each <= 2^-126): O = 0, LSE = -inf
+      const bool dead = (m_use == -INFINITY) || !(lr > 0.f);
+      const float inv = dead ? 0.f : 1.f / lr;
       uint8_t* orow = nullptr;
       if (row_ok) {
         const int64_t ro = varlen ? static_cast<int64_t>(q0 + i) * p.o_ss
@@ -438,7 +553,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       if (row_ok && p.lse != nullptr) {
-        const float lse = (l > 0.f) ? (m_use + __log2f(l)) * kLn2 : -INFINITY;
+        const float lse = dead ? -INFINITY : (m_use + __log2f(l)) * kLn2;
         const int64_t li = varlen ? static_cast<int64_t>(h) * p.total_q + q0 + i
                                   : (static_cast<int64_t>(b) * p.H + h) * p.Sq + i;
         p.lse[li] = lse;

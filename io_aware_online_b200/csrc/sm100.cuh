@@ -107,6 +107,17 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Plain (non-tensor) bulk copy global -> this CTA's shared memory; both addresses
+// 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2) {
   asm volatile(
@@ -137,11 +148,12 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far is done.
+// (No "memory" clobber on the MMA-side asm: their order is kept by asm volatile, and
+// a clobber would make the single issuing thread reload its state after every MMA.)
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
+          smem_u32(bar)));
 }
 
 // D(tmem) (+)= A(smem desc) * B(smem desc)
@@ -151,8 +163,7 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // D(tmem) (+)= A(tmem) * B(smem desc)
@@ -162,8 +173,7 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled tile (sm_100 format:
@@ -178,6 +188,14 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
   return d;
+}
+
+// The same descriptor advanced by `bytes` (a multiple of 16).  Only the 14-bit
+// start-address field changes, and it cannot carry: shared memory addresses are
+// below 256 KiB.  One 32-bit add on the low word.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+  const uint32_t lo = static_cast<uint32_t>(desc) + (bytes >> 4);
+  return (desc & 0xFFFFFFFF00000000ull) | lo;
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16 with fp32 accumulation.
@@ -290,6 +308,38 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
       : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
         "l"(*reinterpret_cast<uint64_t*>(&c)));
   return *reinterpret_cast<float2*>(&r);
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Base-2 exponential of a pair of arguments on the FMA pipe (leaves the MUFU
+// unit to other work).  x = j + f with j = round(x) and f in [-1/2, 1/2]; 2^f is
+// the degree-3 polynomial whose maximum relative error on [-1/2, 1/2] is minimal
+// (Remez exchange; 7.5e-5; coefficients from gen_exp2_poly.py), and 2^j is added
+// to its exponent field.  Valid for x <= 126; arguments below -126 (including
+// -inf) are clamped and give a value <= 2^-126 instead of 0, so callers detect
+// rows without any allowed key by their running max, not by a zero sum.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound holds round(x) in its low bits
+  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = add2(x, make_float2(kRound, kRound));
+  const float2 j = add2(t, make_float2(-kRound, -kRound));
+  const float2 f = fma2(j, make_float2(-1.f, -1.f), x);
+  float2 p = fma2(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+  p = fma2(p, f, make_float2(kC1, kC1));
+  p = fma2(p, f, make_float2(kC0, kC0));
+  // the low bits of t are j (two's complement); shifted by 23 they land on the
+  // exponent field and every bit of the rounding constant falls off the top
+  const uint32_t rx = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
+  const uint32_t ry = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
+  return make_float2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
 // Two fp32 values rounded to the 16-bit input type, lower index in the low half.

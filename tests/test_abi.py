@@ -108,6 +108,7 @@ def kvc(lib, **kw):
     (dict(nblk=0), FA_ERR_INVALID_ARG),
     (dict(d=80), FA_ERR_UNSUPPORTED),
     (dict(splits=4, ws=None, wsb=0), FA_ERR_WORKSPACE),
+    (dict(splits=1, ws=None, wsb=0), FA_ERR_WORKSPACE),       # the item counter lives there
     (dict(bt=None, skmax=-1), FA_ERR_INVALID_ARG),
 ])
 def test_kvcache_validation(lib, kw, code):
@@ -118,8 +119,8 @@ def test_splits_and_workspace_size(lib):
     # explicit split counts are clamped to the number of pages
     assert lib.fa_kvcache_num_splits(64, 1, 32, 8, 128, 32768, 256, 16) == 16
     assert lib.fa_kvcache_num_splits(64, 1, 32, 8, 128, 512, 256, 16) == 2
-    assert lib.fa_kvcache_workspace_size(64, 1, 32, 8, 128, 32768, 256, 1) == 0
-    assert lib.fa_kvcache_workspace_size(64, 1, 32, 8, 128, 32768, 256, 4) == 4 * 64 * 32 * 129 * 4
+    assert lib.fa_kvcache_workspace_size(64, 1, 32, 8, 128, 32768, 256, 1) == 256
+    assert lib.fa_kvcache_workspace_size(64, 1, 32, 8, 128, 32768, 256, 4) == 256 + 4 * 64 * 32 * 129 * 4
 
 
 def test_combine_validation(lib):
