@@ -158,6 +158,35 @@ FA_API int fa_fwd_kvcache(const void *q, const void *k_cache, const void *v_cach
                    size_t workspace_bytes, void *stream);
 
 /*
+ * fa_fwd_kvcache_static -- fa_fwd_kvcache without a workspace argument, for callers
+ * that cannot allocate device memory where they run attention (a host framework
+ * that owns every device allocation through its own pool, or a serving loop that
+ * must not risk the device synchronisation a cudaMalloc can cause).  The pages
+ * have no counterpart to this call.  It allocates nothing: its scratch (the
+ * work-item counter and the fp32 split partials) is one fixed 16 MiB array in
+ * device memory (fa_kvcache_static_scratch_bytes()), present on every GPU that
+ * loads the library until the process exits.  Arguments and results are those of
+ * fa_fwd_kvcache.  A call whose need (fa_kvcache_workspace_size) exceeds the array
+ * returns FA_ERR_WORKSPACE without launching anything.  All calls share the array
+ * and it keeps the last call's contents; each call clears the counter on its own
+ * stream, so calls that overlap on the GPU race and must be serialised by the
+ * caller.  The first call on a device looks the array's address up
+ * (cudaGetSymbolAddress) with that device current; make it before any stream
+ * capture.
+ */
+FA_API int fa_fwd_kvcache_static(const void *q, const void *k_cache, const void *v_cache,
+                                 void *out, float *lse, int dtype, int batch, int seqlen_q,
+                                 int num_heads, int num_heads_k, int head_dim,
+                                 const int32_t *block_table, int max_blocks_per_seq,
+                                 int page_size, int num_blocks, int seqlen_k_max,
+                                 const int32_t *cache_seqlens, float softmax_scale, int causal,
+                                 int window_left, int window_right, float softcap,
+                                 const float *alibi_slopes, int num_splits, void *stream);
+
+/* Size in bytes of the fixed scratch array behind fa_fwd_kvcache_static. */
+FA_API size_t fa_kvcache_static_scratch_bytes(void);
+
+/*
  * fa_combine -- LSE-weighted combine of split partial results
  * (section 3.4 flash_attn_combine; changelog v2.2: "an extra kernel reduces").
  *   LSE = log sum_s exp(lse_s);  O = sum_s exp(lse_s - LSE) * O_s

@@ -9,6 +9,7 @@ library is missing or a call fails, an exception is raised.
 Functions mirror include/fa.h:
     fa_fwd(q, k, v, ...)                  dense [B,S,H,d] or varlen [total,H,d]
     fa_fwd_kvcache(q, k_cache, v_cache, ...)
+    fa_fwd_kvcache_static(q, k_cache, v_cache, ...)   (no workspace; fixed device scratch)
     fa_combine(out_partial, lse_partial, ...)
     fa_kvcache_num_splits(...), fa_kvcache_workspace_size(...)
     fa_device_status(clear=True), fa_set_wait_timeout_ms(ms), fa_version()
@@ -21,7 +22,8 @@ import os
 
 import torch
 
-__all__ = ["FAError", "fa_fwd", "fa_fwd_kvcache", "fa_combine", "fa_kvcache_num_splits",
+__all__ = ["FAError", "fa_fwd", "fa_fwd_kvcache", "fa_fwd_kvcache_static", "fa_combine",
+           "fa_kvcache_num_splits",
            "fa_kvcache_workspace_size", "fa_device_status", "fa_set_wait_timeout_ms",
            "fa_version", "library_path", "load"]
 
@@ -64,6 +66,12 @@ def load():
                                    i32, i32, vp, f32, i32, i32, i32, f32, vp, i32, vp,
                                    ctypes.c_size_t, vp]
     lib.fa_fwd_kvcache.restype = i32
+    lib.fa_fwd_kvcache_static.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp,
+                                          i32, i32, i32, i32, vp, f32, i32, i32, i32, f32, vp,
+                                          i32, vp]
+    lib.fa_fwd_kvcache_static.restype = i32
+    lib.fa_kvcache_static_scratch_bytes.argtypes = []
+    lib.fa_kvcache_static_scratch_bytes.restype = ctypes.c_size_t
     lib.fa_combine.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64p, i64p, vp]
     lib.fa_combine.restype = i32
     lib.fa_last_error.argtypes = []
@@ -221,6 +229,38 @@ def fa_fwd_kvcache(q, k_cache, v_cache, *, cache_seqlens=None, block_table=None,
                               int(bool(causal)), int(window_size[0]), int(window_size[1]),
                               float(softcap), _ptr(alibi_slopes), int(num_splits),
                               _ptr(workspace), ws_bytes, _stream(stream)))
+    return out, lse
+
+
+def fa_fwd_kvcache_static(q, k_cache, v_cache, *, cache_seqlens=None, block_table=None,
+                          softmax_scale=None, causal=False, window_size=(-1, -1), softcap=0.0,
+                          alibi_slopes=None, num_splits=0, out=None, lse=None,
+                          return_lse=True, stream=None):
+    """fa_fwd_kvcache for callers that cannot allocate device memory at the call:
+    the scratch comes from the library's fixed device array (see include/fa.h).
+    Outputs not passed in are allocated here by torch, before the call."""
+    lib = load()
+    dt = _dtype(q)
+    B, sq, H, d = q.shape
+    for t in (q, k_cache, v_cache):
+        if not t.is_contiguous():
+            raise ValueError("q and the caches must be contiguous")
+    if block_table is not None:
+        num_blocks, page, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+        max_blocks, sk_max = block_table.shape[1], 0
+    else:
+        num_blocks, page, max_blocks = 0, 0, 0
+        sk_max, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, sq), dtype=torch.float32, device=q.device)
+    _check(lib.fa_fwd_kvcache_static(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
+                                     dt, B, sq, H, Hkv, d, _ptr(block_table), max_blocks, page,
+                                     num_blocks, sk_max, _ptr(cache_seqlens),
+                                     _scale(softmax_scale), int(bool(causal)),
+                                     int(window_size[0]), int(window_size[1]), float(softcap),
+                                     _ptr(alibi_slopes), int(num_splits), _stream(stream)))
     return out, lse
 
 

@@ -175,6 +175,11 @@ int resolve_splits(int batch, int Sq, int H, int Hkv, int d, int max_seqlen_k, i
 
 }  // namespace
 
+namespace fa {
+// Error reporting for entry points defined in other translation units.
+int set_error(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace fa
+
 extern "C" {
 
 const char* fa_last_error(void) { return g_err.c_str(); }

@@ -71,4 +71,7 @@ struct CombineParams {
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
+// Sets the calling thread's fa_last_error() message; returns `code`.
+int set_error(int code, const char* msg);
+
 }  // namespace fa
