@@ -11,20 +11,22 @@
 //   warps 0-3  softmax warpgroup of tile 0 (thread r owns query row r = TMEM lane r)
 //   warps 4-7  softmax warpgroup of tile 1
 //   warp  8    TMA producer: Q once, then K_j / V_j blocks into a ring of stages
-//   warp  9    tensor-memory allocator and single-thread tcgen05.mma issuer
-//   warps 10-11 idle (they complete the third warpgroup for the register re-split:
+//   warps 9-10 tcgen05.mma issuers, one per query tile (one elected thread each),
+//              so the two tiles' QK/PV chains never wait on each other; warp 9 also
+//              allocates tensor memory
+//   warp  11   idle (it completes the third warpgroup for the register re-split:
 //              the softmax warpgroups hold a 128-float score row per thread and
 //              take 200 registers; the third warpgroup keeps 104)
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   S_t = Q_t K_j^T   at columns [128 t, 128 t + 128)        (t = 0, 1)
 //   P_t (16-bit)      aliases the first 64 columns of S_t (two values per column)
 //   O_t += P_t V_j    at columns [256 + D t, 256 + D t + D)
-// The MMA warp alternates the two tiles (ping-pong) so that the softmax of one
-// tile overlaps the tensor-core work of the other:
-//   PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1)
-// Each commit to S_t's barrier also covers the PV_t(j) issued before it, so when
-// a softmax warpgroup sees S_t(j+1) it knows P_t(j) has been consumed and O_t is
-// up to date; it may then rescale O_t in tensor memory before releasing P_t(j+1).
+// Each tile's issuer runs its own chain; with P aliasing S (D = 128) it is
+//   PV_t(j), QK_t(j+1)
+// and each commit to S_t's barrier also covers the PV_t(j) issued before it, so
+// when a softmax warpgroup sees S_t(j+1) it knows P_t(j) has been consumed and O_t
+// is up to date; it may then rescale O_t before releasing P_t(j+1).  With separate
+// P columns (D = 64) QK_t(j+1) is issued as soon as S_t(j) sits in registers.
 // The running max is kept lazily: O is rescaled only when a row's max grows by
 // more than 8 (base-2 units); the final O / l and LSE use the same stale max, so
 // the result is unchanged.  Blocks that lie fully inside every row's allowed key
@@ -59,8 +61,8 @@ struct FwdCfg {
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
-  // o_final[2], drain, s_free[2], pv_done[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 11;
+  // o_final[2], drain[2], s_free[2], pv_done[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 12;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // room to align the base to 1 KiB
@@ -163,9 +165,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* s_full = bars + 1 + 4 * ST;
   uint64_t* p_full = bars + 3 + 4 * ST;
   uint64_t* o_final = bars + 5 + 4 * ST;
-  uint64_t* drain = bars + 7 + 4 * ST;
-  uint64_t* s_free = bars + 8 + 4 * ST;   // softmax has S_t in registers (separate-P layout)
-  uint64_t* pv_done = bars + 10 + 4 * ST; // PV_t finished: P_t may be rewritten, O_t rescaled
+  uint64_t* drain = bars + 7 + 4 * ST;    // [2]: one per issuer
+  uint64_t* s_free = bars + 9 + 4 * ST;   // softmax has S_t in registers (separate-P layout)
+  uint64_t* pv_done = bars + 11 + 4 * ST; // PV_t finished: P_t may be rewritten, O_t rescaled
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -173,9 +175,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < ST; ++s) {
       mbar_init(k_full + s, 1);
-      mbar_init(k_empty + s, 1);
+      mbar_init(k_empty + s, 2);  // released by both issuers
       mbar_init(v_full + s, 1);
-      mbar_init(v_empty + s, 1);
+      mbar_init(v_empty + s, 2);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full + t, 1);
@@ -184,7 +186,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(s_free + t, kBM);
       mbar_init(pv_done + t, 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain + 0, 1);
+    mbar_init(drain + 1, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -242,117 +245,121 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
     __syncwarp();
-   } else if (warp == 9) {
-    // ======================================================== MMA issuer
+   } else if (warp == 9 && !Cfg::kSepP) {
+    // ======================================================== MMA issuer (D = 128)
+    // One thread alternates the tiles, PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): the
+    // two softmax warpgroups then take turns on the exponential unit.
     if (lane == 0 && n_blk > 0) {
       constexpr uint32_t idesc_qk = f16_idesc(BF16, kBM, kBN, false, false);
       constexpr uint32_t idesc_pv = f16_idesc(BF16, kBM, D, false, true);
-      // Descriptor bases computed once; every MMA below forms its operand
-      // descriptors with one add on the low word (the issuing thread is on the
-      // critical path of the pipeline, so its per-instruction work stays small).
-      const uint64_t dQ = sw128_desc(smem_u32(sQ), 16, 1024);               // K-major
-      const uint64_t dK = sw128_desc(smem_u32(sK), 16, 1024);               // K-major
-      const uint64_t dV = sw128_desc(smem_u32(sV), Cfg::kChunkBytes, 1024); // MN-major
-      const uint32_t tS0 = tbase, tS1 = tbase + kBM;
-      const uint32_t tP0 = tbase + Cfg::kPCol, tP1 = tbase + Cfg::kPCol + Cfg::kPStride;
-      const uint32_t tO0 = tbase + Cfg::kOCol, tO1 = tbase + Cfg::kOCol + D;
-      const uint64_t dQ0 = dQ, dQ1 = desc_advance(dQ, Cfg::kTileBytes);
-#define FA_QK(T, S)                                                                         \
-  fwd_issue_qk<D>(T ? tS1 : tS0, T ? dQ1 : dQ0, desc_advance(dK, (S) * Cfg::kTileBytes),   \
-                  idesc_qk)
-#define FA_PV(T, S, ACC)                                                                    \
-  fwd_issue_pv<D>(T ? tO1 : tO0, T ? tP1 : tP0, desc_advance(dV, (S) * Cfg::kTileBytes),   \
-                  idesc_pv, ACC)
-#define qk(T, S) FA_QK(T, S)
-#define pv(T, S, ACC) FA_PV(T, S, ACC)
+      const uint64_t dQ0 = sw128_desc(smem_u32(sQ), 16, 1024);
+      const uint64_t dQ1 = desc_advance(dQ0, Cfg::kTileBytes);
+      const uint64_t dK = sw128_desc(smem_u32(sK), 16, 1024);
+      const uint64_t dV = sw128_desc(smem_u32(sV), Cfg::kChunkBytes, 1024);
+#define FA_QK(T, S)                                                                    \
+  fwd_issue_qk<D>(tbase + (T) * kBM, (T) ? dQ1 : dQ0,                                    \
+                  desc_advance(dK, (S) * Cfg::kTileBytes), idesc_qk)
+#define FA_PV(T, S, ACC)                                                               \
+  fwd_issue_pv<D>(tbase + Cfg::kOCol + (T) * D, tbase + Cfg::kPCol + (T) * Cfg::kPStride, \
+                  desc_advance(dV, (S) * Cfg::kTileBytes), idesc_pv, ACC)
       bool ok = wait_bounded(q_full, 0, w) && wait_bounded(k_full, 0, w);
-      if (ok && Cfg::kSepP) {
-        // QK_t(j+1) as soon as softmax t holds S_t(j) in registers; PV_t(j) when P_t(j)
-        // is written.  Each tile's softmax then runs back to back.
+      if (ok) {
         tc_fence_after();
-        qk(0, 0);
+        FA_QK(0, 0);
         tc_commit(s_full + 0);
-        qk(1, 0);
+        FA_QK(1, 0);
         tc_commit(s_full + 1);
         tc_commit(k_empty + 0);
-        for (int it = 0; it < n_blk && ok; ++it) {
-          const int s = it % ST;
-          const uint32_t ph = (it / ST) & 1;
-          const bool more = it + 1 < n_blk;
-          const int s1 = (it + 1) % ST;
-          const uint32_t ph1 = ((it + 1) / ST) & 1;
-          if (more) {
-            if (!(ok = wait_bounded(k_full + s1, ph1, w))) break;
-            if (!(ok = wait_bounded(s_free + 0, it & 1, w))) break;
-            tc_fence_after();
-            qk(0, s1);
-            tc_commit(s_full + 0);
-          }
-          if (!(ok = wait_bounded(v_full + s, ph, w))) break;
-          if (!(ok = wait_bounded(p_full + 0, it & 1, w))) break;
+        tc_commit(k_empty + 0);  // k_empty counts one release per tile
+      }
+      for (int it = 0; it < n_blk && ok; ++it) {
+        const int s = it % ST;
+        const uint32_t ph = (it / ST) & 1;
+        const bool more = it + 1 < n_blk;
+        const int s1 = (it + 1) % ST;
+        const uint32_t ph1 = ((it + 1) / ST) & 1;
+        if (!(ok = wait_bounded(v_full + s, ph, w))) break;
+        if (!(ok = wait_bounded(p_full + 0, it & 1, w))) break;
+        tc_fence_after();
+        FA_PV(0, s, it > 0);
+        tc_commit(v_empty + s);
+        if (more) {
+          if (!(ok = wait_bounded(k_full + s1, ph1, w))) break;
           tc_fence_after();
-          pv(0, s, it > 0);
-          tc_commit(pv_done + 0);
-          if (!more) tc_commit(o_final + 0);
-          if (more) {
-            if (!(ok = wait_bounded(s_free + 1, it & 1, w))) break;
-            tc_fence_after();
-            qk(1, s1);
-            tc_commit(s_full + 1);
-            tc_commit(k_empty + s1);
-          }
-          if (!(ok = wait_bounded(p_full + 1, it & 1, w))) break;
-          tc_fence_after();
-          pv(1, s, it > 0);
-          tc_commit(pv_done + 1);
-          tc_commit(v_empty + s);
-          if (!more) tc_commit(o_final + 1);
+          FA_QK(0, s1);
+          tc_commit(s_full + 0);
+          tc_commit(k_empty + s1);
+        } else {
+          tc_commit(o_final + 0);
         }
-      } else if (ok) {
+        if (!(ok = wait_bounded(p_full + 1, it & 1, w))) break;
         tc_fence_after();
-        qk(0, 0);
-        tc_commit(s_full + 0);
-        qk(1, 0);
-        tc_commit(s_full + 1);
-        tc_commit(k_empty + 0);
-        for (int it = 0; it < n_blk && ok; ++it) {
-          const int s = it % ST;
-          const uint32_t ph = (it / ST) & 1;
-          const bool more = it + 1 < n_blk;
-          const int s1 = (it + 1) % ST;
-          const uint32_t ph1 = ((it + 1) / ST) & 1;
-          if (!(ok = wait_bounded(v_full + s, ph, w))) break;
-          if (!(ok = wait_bounded(p_full + 0, it & 1, w))) break;
-          tc_fence_after();
-          pv(0, s, it > 0);
-          if (more) {
-            if (!(ok = wait_bounded(k_full + s1, ph1, w))) break;
-            tc_fence_after();
-            qk(0, s1);
-            tc_commit(s_full + 0);
-          } else {
-            tc_commit(o_final + 0);
-          }
-          if (!(ok = wait_bounded(p_full + 1, it & 1, w))) break;
-          tc_fence_after();
-          pv(1, s, it > 0);
-          tc_commit(v_empty + s);
-          if (more) {
-            qk(1, s1);
-            tc_commit(s_full + 1);
-            tc_commit(k_empty + s1);
-          } else {
-            tc_commit(o_final + 1);
-          }
+        FA_PV(1, s, it > 0);
+        tc_commit(v_empty + s);
+        if (more) {
+          FA_QK(1, s1);
+          tc_commit(s_full + 1);
+          tc_commit(k_empty + s1);
+        } else {
+          tc_commit(o_final + 1);
         }
       }
-#undef qk
-#undef pv
+#undef FA_QK
+#undef FA_PV
+      tc_commit(drain + 0);
+      wait_drain(drain + 0, 0, p.timeout_ns);
+    }
+    __syncwarp();
+   } else if (Cfg::kSepP && (warp == 9 || warp == 10)) {
+    // ======================================================== MMA issuers (D = 64)
+    const int t = warp - 9;  // this issuer's query tile
+    if (lane == 0 && n_blk > 0) {
+      constexpr uint32_t idesc_qk = f16_idesc(BF16, kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = f16_idesc(BF16, kBM, D, false, true);
+      const uint32_t tS = tbase + t * kBM;
+      const uint32_t tP = tbase + Cfg::kPCol + t * Cfg::kPStride;
+      const uint32_t tO = tbase + Cfg::kOCol + t * D;
+      const uint64_t dQ = desc_advance(sw128_desc(smem_u32(sQ), 16, 1024), t * Cfg::kTileBytes);
+      const uint64_t dK = sw128_desc(smem_u32(sK), 16, 1024);               // K-major
+      const uint64_t dV = sw128_desc(smem_u32(sV), Cfg::kChunkBytes, 1024); // MN-major
+#define FA_QK(S) fwd_issue_qk<D>(tS, dQ, desc_advance(dK, (S) * Cfg::kTileBytes), idesc_qk)
+#define FA_PV(S, ACC) \
+  fwd_issue_pv<D>(tO, tP, desc_advance(dV, (S) * Cfg::kTileBytes), idesc_pv, ACC)
+      bool ok = wait_bounded(q_full, 0, w) && wait_bounded(k_full, 0, w);
+      if (ok) {
+        tc_fence_after();
+        FA_QK(0);
+        tc_commit(s_full + t);
+        tc_commit(k_empty + 0);
+      }
+      for (int it = 0; it < n_blk && ok; ++it) {
+        const int s = it % ST;
+        const uint32_t ph = (it / ST) & 1;
+        const bool more = it + 1 < n_blk;
+        const int s1 = (it + 1) % ST;
+        const uint32_t ph1 = ((it + 1) / ST) & 1;
+        // QK_t(j+1) as soon as softmax t holds S_t(j) in registers
+        if (more) {
+          if (!(ok = wait_bounded(k_full + s1, ph1, w))) break;
+          if (!(ok = wait_bounded(s_free + t, it & 1, w))) break;
+          tc_fence_after();
+          FA_QK(s1);
+          tc_commit(s_full + t);
+          tc_commit(k_empty + s1);
+        }
+        if (!(ok = wait_bounded(v_full + s, ph, w))) break;
+        if (!(ok = wait_bounded(p_full + t, it & 1, w))) break;
+        tc_fence_after();
+        FA_PV(s, it > 0);
+        tc_commit(pv_done + t);
+        tc_commit(v_empty + s);
+        if (!more) tc_commit(o_final + t);
+      }
 #undef FA_QK
 #undef FA_PV
       // every MMA issued above is complete before tensor memory is released
-      tc_commit(drain);
-      wait_drain(drain, 0, p.timeout_ns);
+      tc_commit(drain + t);
+      wait_drain(drain + t, 0, p.timeout_ns);
     }
     __syncwarp();
    }
@@ -452,24 +459,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         l *= alpha;
         lr *= alpha;
       }
-      // ---- probabilities -> 16-bit P in tensor memory
-      if constexpr (Cfg::kSepP) {
-        // P_t(j-1) must have been consumed (and O_t updated) by PV_t(j-1)
-        if (it > 0) {
-          ok = wait_bounded(pv_done + t, (it - 1) & 1, w);
-          if (!__all_sync(0xffffffffu, ok)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-        }
-      }
+      // ---- probabilities -> 16-bit P in tensor memory.  With separate P columns
+      // the whole row is computed first and the wait for PV_t(j-1) (which still
+      // reads P_t) comes only before the stores, so the exponentials overlap it.
       const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
       const float2 f2 = make_float2(factor, factor), nm2 = make_float2(neg_m, neg_m);
       float2 lsum[kBN / 32], lrnd[kBN / 32];
+      uint32_t pk[kBN / 2];
 #pragma unroll
       for (int q4 = 0; q4 < kBN / 32; ++q4) {
-        uint32_t pk[16];
         lsum[q4] = make_float2(0.f, 0.f);
         lrnd[q4] = make_float2(0.f, 0.f);
 #pragma unroll
@@ -482,13 +480,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             pp = exp2_fma2(arg);
           else
             pp = make_float2(ex2(arg.x), ex2(arg.y));
-          pk[e] = pack2<BF16>(pp.x, pp.y);
+          pk[q4 * 16 + e] = pack2<BF16>(pp.x, pp.y);
           lsum[q4] = add2(lsum[q4], pp);
           // bf16 P is rounded by up to 2^-9: sum the rounded values the PV product
           // uses, so that O / lr is an exact convex combination of V rows
-          if constexpr (BF16) lrnd[q4] = add2(lrnd[q4], unpack2<true>(pk[e]));
+          if constexpr (BF16) lrnd[q4] = add2(lrnd[q4], unpack2<true>(pk[q4 * 16 + e]));
         }
-        tmem_st16(tP + q4 * 16, pk);
+        if constexpr (!Cfg::kSepP) tmem_st16(tP + q4 * 16, pk + q4 * 16);
+      }
+      if constexpr (Cfg::kSepP) {
+        // P_t(j-1) must have been consumed (and O_t updated) by PV_t(j-1)
+        if (it > 0) {
+          ok = wait_bounded(pv_done + t, (it - 1) & 1, w);
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < kBN / 32; ++q4) tmem_st16(tP + q4 * 16, pk + q4 * 16);
       }
       {
         float2 a = add2(add2(lsum[0], lsum[1]), add2(lsum[2], lsum[3]));

@@ -29,7 +29,7 @@ inline int exp2_emu_choice(int d) {
     return e ? std::atoi(e) : -1;
   }();
   if (env == 0 || env == 2 || env == 3 || env == 4) return env;
-  return d == 64 ? 3 : 0;
+  return d == 64 ? 2 : 0;
 }
 
 template <bool BF16>
