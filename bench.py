@@ -49,6 +49,26 @@ def prefill_flops(c=PREFILL) -> float:
     return 4.0 * c["d"] * c["B"] * c["H"] * causal_pairs(c["S"], c["S"])
 
 
+def profiled_traffic(profile: str, sources) -> int | None:
+    """DRAM bytes per launch from a committed ncu summary, or None when the kernel's
+    sources no longer hash to the value recorded with the capture."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", profile)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_t = re.search(r"^traffic_bytes_per_launch: (\d+)", text, re.M)
+    m_h = re.search(r"^source_sha256_16: ([0-9a-f]+)", text, re.M)
+    if not (m_t and m_h):
+        return None
+    h = hashlib.sha256()
+    for f in sources:
+        with open(os.path.join(ROOT, "io_aware_online_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return int(m_t.group(1)) if h.hexdigest()[:16] == m_h.group(1) else None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -278,12 +298,19 @@ def run_ours(args, rank, world, local):
             "roofline": {"bound": "hbm", "achieved": round(dbytes / (t_dec_max * 1e-3) / 1e9, 1),
                          "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(dbytes / (t_dec_max * 1e-3) / 1e9 / hbm_peak, 4),
-                         "traffic": None, "peak_source": peak_src},
+                         "traffic": (profiled_traffic("decode_kernel_paged_B8.md",
+                                                      ["decode_kernel.cuh", "decode.cu",
+                                                       "sm100.cuh", "fa_internal.h"])
+                                     if (DECODE["B"] == 64 and splits == 16) else None),
+                         "peak_source": peak_src},
         },
         "roofline": {"bound": "tensor", "achieved": round(flops / (t_pre * 1e-3) / 1e12, 2),
                      "peak": tflops_peak, "unit": "TFLOP/s",
                      "frac": round(flops / (t_pre * 1e-3) / 1e12 / tflops_peak, 4),
-                     "traffic": None,
+                     "traffic": (profiled_traffic("fwd_kernel_d64_causal_B4_S4096.md",
+                                                  ["fwd_kernel.cuh", "fwd_launch.cuh",
+                                                   "sm100.cuh", "fa_internal.h"])
+                                 if (PREFILL["d"] == 64 and PREFILL["S"] == 4096) else None),
                      "kernel": f"fwd_kernel<{PREFILL['d']}, {PREFILL['dtype']}, causal>",
                      "peak_source": f"{peak_src} bf16 burst (fp16 dense rate equals bf16)"},
         "gpu_launches": K * ((1 if do_pre else 0) + ((2 if splits > 1 else 1) if do_dec else 0)),
