@@ -61,8 +61,8 @@ struct FwdCfg {
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
-  // o_final[2], drain[2], s_free[2], pv_done[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 12;
+  // o_final[2], drain[2], s_free[2], pv_done[2], turn[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 14;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // room to align the base to 1 KiB
@@ -168,6 +168,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* drain = bars + 7 + 4 * ST;    // [2]: one per issuer
   uint64_t* s_free = bars + 9 + 4 * ST;   // softmax has S_t in registers (separate-P layout)
   uint64_t* pv_done = bars + 11 + 4 * ST; // PV_t finished: P_t may be rewritten, O_t rescaled
+  uint64_t* turn = bars + 13 + 4 * ST;    // exponential-phase handoff between the warpgroups
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -181,10 +182,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full + t, 1);
-      mbar_init(p_full + t, kBM);
+      mbar_init(p_full + t, 4);   // one arrival per softmax warp
       mbar_init(o_final + t, 1);
-      mbar_init(s_free + t, kBM);
+      mbar_init(s_free + t, 4);
       mbar_init(pv_done + t, 1);
+      mbar_init(turn + t, 4);  // one arrival per warp of the other warpgroup
     }
     mbar_init(drain + 0, 1);
     mbar_init(drain + 1, 1);
@@ -399,7 +401,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int c = 0; c < kBN / 32; ++c) tmem_ld_wait(s + c * 32);
       if constexpr (Cfg::kSepP) {  // S_t may now be overwritten by the next QK
         tc_fence_before();
-        mbar_arrive(s_free + t);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free + t);
       }
 
       const bool masked = (kb < lo_rb) || (kb + kBN - 1 > hi_ra);
@@ -462,6 +465,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // ---- probabilities -> 16-bit P in tensor memory.  With separate P columns
       // the whole row is computed first and the wait for PV_t(j-1) (which still
       // reads P_t) comes only before the stores, so the exponentials overlap it.
+      // The two warpgroups take turns for this exponential phase (tile 0 first), so
+      // one's exponentials run while the other loads and reduces its next row and
+      // the MUFU unit stays busy instead of being shared half of the time and idle
+      // the other half.  Pure scheduling: results do not depend on it.
+      if (p.turns && (t == 1 || it > 0)) {
+        ok = wait_bounded(turn + t, (t == 0 ? it - 1 : it) & 1, w);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+      }
       const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
       const float2 f2 = make_float2(factor, factor), nm2 = make_float2(neg_m, neg_m);
       float2 lsum[kBN / 32], lrnd[kBN / 32];
@@ -488,6 +502,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         if constexpr (!Cfg::kSepP) tmem_st16(tP + q4 * 16, pk + q4 * 16);
       }
+      __syncwarp();
+      if (p.turns && lane == 0) mbar_arrive(turn + (1 - t));  // hand the exponential unit over
       if constexpr (Cfg::kSepP) {
         // P_t(j-1) must have been consumed (and O_t updated) by PV_t(j-1)
         if (it > 0) {
@@ -522,7 +538,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full + t);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full + t);
     }
 
     // ---- epilogue: O / l -> 16-bit, LSE (natural log)
