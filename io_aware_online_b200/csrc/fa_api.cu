@@ -296,13 +296,6 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
   p.wr = window_right;
   p.status = status;
   p.timeout_ns = timeout_ns();
-  {
-    static const int turns_env = [] {
-      const char* e = std::getenv("FA_SOFTMAX_TURNS");
-      return e ? std::atoi(e) : -1;
-    }();
-    p.turns = turns_env >= 0 ? (turns_env != 0) : 0;
-  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = (dtype == FA_BF16)
                       ? fa::launch_fwd_bf16(tq, tk, tv, p, d, batch, n_pairs, st)

@@ -25,7 +25,6 @@ struct FwdParams {
   int causal, wl, wr;              // mask flags; -1 = unbounded window side
   unsigned int* status;            // device status word
   uint64_t timeout_ns;             // bounded-wait limit
-  int turns;                       // softmax warpgroups alternate their exponential phases
 };
 
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

@@ -34,6 +34,7 @@
 #pragma once
 
 #include <climits>
+#include <type_traits>
 
 #include "fa_internal.h"
 #include "sm100.cuh"
@@ -61,8 +62,8 @@ struct FwdCfg {
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
-  // o_final[2], drain[2], s_free[2], pv_done[2], turn[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 14;
+  // o_final[2], drain[2], s_free[2], pv_done[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 12;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // room to align the base to 1 KiB
@@ -168,7 +169,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* drain = bars + 7 + 4 * ST;    // [2]: one per issuer
   uint64_t* s_free = bars + 9 + 4 * ST;   // softmax has S_t in registers (separate-P layout)
   uint64_t* pv_done = bars + 11 + 4 * ST; // PV_t finished: P_t may be rewritten, O_t rescaled
-  uint64_t* turn = bars + 13 + 4 * ST;    // exponential-phase handoff between the warpgroups
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -186,7 +186,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(o_final + t, 1);
       mbar_init(s_free + t, 4);
       mbar_init(pv_done + t, 1);
-      mbar_init(turn + t, 4);  // one arrival per warp of the other warpgroup
     }
     mbar_init(drain + 0, 1);
     mbar_init(drain + 1, 1);
@@ -249,8 +248,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncwarp();
    } else if (warp == 9 && !Cfg::kSepP) {
     // ======================================================== MMA issuer (D = 128)
-    // One thread alternates the tiles, PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): the
-    // two softmax warpgroups then take turns on the exponential unit.
+    // One thread alternates the tiles, PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so
+    // one tile's softmax overlaps the other tile's products.
     if (lane == 0 && n_blk > 0) {
       constexpr uint32_t idesc_qk = f16_idesc(BF16, kBM, kBN, false, false);
       constexpr uint32_t idesc_pv = f16_idesc(BF16, kBM, D, false, true);
@@ -436,74 +435,89 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         factor = 1.f;
       }
-      // ---- row max: four independent chains of three-input max
-      float m_blk;
-      {
-        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < kBN; c += 8) {
-          a0 = max3f(a0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-          a1 = max3f(a1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
-          a2 = max3f(a2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
-          a3 = max3f(a3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
-        }
-        m_blk = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * factor;
-      }
-      // ---- online softmax bookkeeping (lazy rescale)
-      const float m_new = fmaxf(m_use, m_blk);
+      // ---- row max, online-softmax bookkeeping (lazy rescale), exponentials.
+      // With P aliasing S (D = 128) the exponentials are taken speculatively
+      // against the running max while the block's row max is reduced in the same
+      // loop.  If no row's max grew by more than the rescale threshold, the running
+      // max stays as it is and the probabilities are exactly those of the max-first
+      // order; otherwise the warp takes the exponentials again against the new max
+      // (rows whose max did not move recompute the same values).  The raw scores
+      // stay in registers until that check.  Warps with a row that has not met an
+      // allowed key yet (running max -inf) take the max-first order.
+      const bool spec = !Cfg::kSepP && __all_sync(0xffffffffu, m_use != -INFINITY);
       bool need = false;
       float alpha = 1.f;
-      if (m_use == -INFINITY) {
-        m_use = m_new;  // nothing accumulated yet: O is zero
-      } else if (m_new > m_use + kRescaleThreshold) {
-        need = true;
-        alpha = ex2(m_use - m_new);
-        m_use = m_new;
-        l *= alpha;
-        lr *= alpha;
-      }
-      // ---- probabilities -> 16-bit P in tensor memory.  With separate P columns
-      // the whole row is computed first and the wait for PV_t(j-1) (which still
-      // reads P_t) comes only before the stores, so the exponentials overlap it.
-      // The two warpgroups take turns for this exponential phase (tile 0 first), so
-      // one's exponentials run while the other loads and reduces its next row and
-      // the MUFU unit stays busy instead of being shared half of the time and idle
-      // the other half.  Pure scheduling: results do not depend on it.
-      if (p.turns && (t == 1 || it > 0)) {
-        ok = wait_bounded(turn + t, (t == 0 ? it - 1 : it) & 1, w);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
+      auto update_max = [&](float m_blk) {
+        const float m_new = fmaxf(m_use, m_blk);
+        if (m_use == -INFINITY) {
+          m_use = m_new;  // nothing accumulated yet: O is zero
+        } else if (m_new > m_use + kRescaleThreshold) {
+          need = true;
+          alpha = ex2(m_use - m_new);
+          m_use = m_new;
         }
+      };
+      // four independent chains of three-input max
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      if (!spec) {
+#pragma unroll
+        for (int c = 0; c < kBN; c += 8) {
+          mx0 = max3f(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+          mx1 = max3f(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+          mx2 = max3f(mx2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+          mx3 = max3f(mx3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+        }
+        update_max(fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * factor);
       }
-      const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
-      const float2 f2 = make_float2(factor, factor), nm2 = make_float2(neg_m, neg_m);
+      // probabilities -> 16-bit P.  With separate P columns the whole row is held
+      // and the wait for PV_t(j-1) (which still reads P_t) comes only before the
+      // stores, so the exponentials overlap it; with P aliasing S each 32-column
+      // chunk is stored as soon as it is ready.
       float2 lsum[kBN / 32], lrnd[kBN / 32];
-      uint32_t pk[kBN / 2];
+      uint32_t pk[Cfg::kSepP ? kBN / 2 : 16];
+      auto exps = [&](auto with_max) {
+        constexpr bool kMax = decltype(with_max)::value;
+        const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+        const float2 f2 = make_float2(factor, factor), nm2 = make_float2(neg_m, neg_m);
 #pragma unroll
-      for (int q4 = 0; q4 < kBN / 32; ++q4) {
-        lsum[q4] = make_float2(0.f, 0.f);
-        lrnd[q4] = make_float2(0.f, 0.f);
+        for (int q4 = 0; q4 < kBN / 32; ++q4) {
+          lsum[q4] = make_float2(0.f, 0.f);
+          lrnd[q4] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float2 arg = fma2(make_float2(__uint_as_float(s[q4 * 32 + 2 * e]),
-                                              __uint_as_float(s[q4 * 32 + 2 * e + 1])),
-                                  f2, nm2);
-          float2 pp;
-          if ((e % 8) < EMU)
-            pp = exp2_fma2(arg);
-          else
-            pp = make_float2(ex2(arg.x), ex2(arg.y));
-          pk[q4 * 16 + e] = pack2<BF16>(pp.x, pp.y);
-          lsum[q4] = add2(lsum[q4], pp);
-          // bf16 P is rounded by up to 2^-9: sum the rounded values the PV product
-          // uses, so that O / lr is an exact convex combination of V rows
-          if constexpr (BF16) lrnd[q4] = add2(lrnd[q4], unpack2<true>(pk[q4 * 16 + e]));
+          for (int e = 0; e < 16; ++e) {
+            const float s0 = __uint_as_float(s[q4 * 32 + 2 * e]);
+            const float s1 = __uint_as_float(s[q4 * 32 + 2 * e + 1]);
+            if constexpr (kMax) {
+              if (e % 4 == 0) mx0 = max3f(mx0, s0, s1);
+              if (e % 4 == 1) mx1 = max3f(mx1, s0, s1);
+              if (e % 4 == 2) mx2 = max3f(mx2, s0, s1);
+              if (e % 4 == 3) mx3 = max3f(mx3, s0, s1);
+            }
+            const float2 arg = fma2(make_float2(s0, s1), f2, nm2);
+            float2 pp;
+            if ((e % 8) < EMU)
+              pp = exp2_fma2(arg);
+            else
+              pp = make_float2(ex2(arg.x), ex2(arg.y));
+            const int pi = Cfg::kSepP ? q4 * 16 + e : e;
+            pk[pi] = pack2<BF16>(pp.x, pp.y);
+            lsum[q4] = add2(lsum[q4], pp);
+            // bf16 P is rounded by up to 2^-9: sum the rounded values the PV product
+            // uses, so that O / lr is an exact convex combination of V rows
+            if constexpr (BF16) lrnd[q4] = add2(lrnd[q4], unpack2<true>(pk[pi]));
+          }
+          if constexpr (!Cfg::kSepP) tmem_st16(tP + q4 * 16, pk);
         }
-        if constexpr (!Cfg::kSepP) tmem_st16(tP + q4 * 16, pk + q4 * 16);
+      };
+      if (spec) {
+        exps(std::true_type{});
+        update_max(fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * factor);
+        if (__any_sync(0xffffffffu, need)) exps(std::false_type{});
+      } else {
+        exps(std::false_type{});
       }
-      __syncwarp();
-      if (p.turns && lane == 0) mbar_arrive(turn + (1 - t));  // hand the exponential unit over
+      l *= alpha;
+      lr *= alpha;
       if constexpr (Cfg::kSepP) {
         // P_t(j-1) must have been consumed (and O_t updated) by PV_t(j-1)
         if (it > 0) {

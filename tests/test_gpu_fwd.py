@@ -114,6 +114,22 @@ def test_softcap_alibi(dtype, d, softcap, alibi, causal):
             window_size=(200, -1) if causal else (-1, -1))
 
 
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16], ids=["fp16", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_max_growing_across_blocks(dtype, d, causal):
+    """Every 128-key block raises each row's max by well over 8 (base 2): the
+    running max is replaced, and O rescaled, at each block (online softmax,
+    FlashAttention-2 section 3.1)."""
+    q, k, v = synth.dense(1, 512, 512, 2, 2, d, dtype, seed=1031)
+    # a shared direction: q . k gains 2 * a_j with a_j = 40 * (j // 128)
+    a = 40.0 * (torch.arange(512) // 128).float()
+    q = (q.float() + 2.0).to(dtype)
+    k = (k.float() + (a / d)[None, :, None, None]).to(dtype)
+    dmax, _ = compare(q, k, v, causal=causal)
+    assert dmax <= ATOL[dtype]
+
+
 def test_more_queries_than_keys_gives_dead_rows():
     q, k, v = synth.dense(1, 300, 100, 2, 2, 64, torch.float16, seed=5)
     compare(q, k, v, causal=True)
