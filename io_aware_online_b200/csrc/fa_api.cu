@@ -246,9 +246,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
       return fail(FA_ERR_INVALID_ARG, "fa_fwd: strides must be positive multiples of 8 elements");
   const int rows_q = varlen ? max_seqlen_q : seqlen_q;
   if (batch == 0 || rows_q == 0) return FA_OK;  // nothing to compute
-  const int n_pairs = (rows_q + 255) / 256;
-  if (batch > 65535 || n_pairs > 65535)
-    return fail(FA_ERR_UNSUPPORTED, "fa_fwd: batch (%d) or query blocks (%d) above 65535", batch, n_pairs);
+  const int n_tiles = (rows_q + 127) / 128;
+  if (batch > 65535 || n_tiles > 65535)
+    return fail(FA_ERR_UNSUPPORTED, "fa_fwd: batch (%d) or query tiles (%d) above 65535", batch, n_tiles);
   if ((rc = get_encoder()) != FA_OK) return rc;
   unsigned int* status = nullptr;
   if ((rc = device_state(nullptr, &status, nullptr)) != FA_OK) return rc;
@@ -298,8 +298,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
   p.timeout_ns = timeout_ns();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = (dtype == FA_BF16)
-                      ? fa::launch_fwd_bf16(tq, tk, tv, p, d, batch, n_pairs, st)
-                      : fa::launch_fwd_f16(tq, tk, tv, p, d, batch, n_pairs, st);
+                      ? fa::launch_fwd_bf16(tq, tk, tv, p, d, batch, rows_q, st)
+                      : fa::launch_fwd_f16(tq, tk, tv, p, d, batch, rows_q, st);
   if (e != cudaSuccess) return cuda_fail(e, "fa_fwd launch");
   return FA_OK;
 }

@@ -27,10 +27,6 @@ struct FwdParams {
   uint64_t timeout_ns;             // bounded-wait limit
 };
 
-cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const FwdParams& p, bool bf16, int d, int batch, int n_pairs,
-                       cudaStream_t stream);
-
 // ---------------------------------------------------------------- decode
 struct DecodeParams {
   const void* q;                   // [B, Sq, H, D] contiguous

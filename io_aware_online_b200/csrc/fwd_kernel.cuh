@@ -7,26 +7,26 @@
 // "FlashAttention common interfaces" sections 3.1/3.2; the causal mask is
 // aligned bottom-right (changelog post, v2.1).
 //
-// CTA = two 128-row query tiles of one (sequence, head); 384 threads:
-//   warps 0-3  softmax warpgroup of tile 0 (thread r owns query row r = TMEM lane r)
-//   warps 4-7  softmax warpgroup of tile 1
-//   warp  8    TMA producer: Q once, then K_j / V_j blocks into a ring of stages
-//   warps 9-10 tcgen05.mma issuers, one per query tile (one elected thread each),
-//              so the two tiles' QK/PV chains never wait on each other; warp 9 also
-//              allocates tensor memory
-//   warp  11   idle (it completes the third warpgroup for the register re-split:
-//              the softmax warpgroups hold a 128-float score row per thread and
-//              take 200 registers; the third warpgroup keeps 104)
-// Tensor memory (512 columns x 128 lanes, fp32):
-//   S_t = Q_t K_j^T   at columns [128 t, 128 t + 128)        (t = 0, 1)
-//   P_t (16-bit)      aliases the first 64 columns of S_t (two values per column)
-//   O_t += P_t V_j    at columns [256 + D t, 256 + D t + D)
-// Each tile's issuer runs its own chain; with P aliasing S (D = 128) it is
-//   PV_t(j), QK_t(j+1)
-// and each commit to S_t's barrier also covers the PV_t(j) issued before it, so
-// when a softmax warpgroup sees S_t(j+1) it knows P_t(j) has been consumed and O_t
-// is up to date; it may then rescale O_t before releasing P_t(j+1).  With separate
-// P columns (D = 64) QK_t(j+1) is issued as soon as S_t(j) sits in registers.
+// CTA = T 128-row query tiles of one (sequence, head), T = 2 (or T = 1 at D = 64,
+// two CTAs per SM); 128 (T + 1) threads:
+//   warps 0 .. 4T-1  softmax warpgroup per tile (thread r owns query row r = TMEM
+//                    lane r of its tile)
+//   warp  4T         TMA producer: Q once, then K_j / V_j blocks into a ring of stages
+//   warp  4T+1 ..    tcgen05.mma issuer(s), one elected thread each; the first also
+//                    allocates tensor memory.  The rest of that warpgroup idles: it
+//                    completes the warpgroup for the register re-split (softmax
+//                    threads hold a 128-float score row and take 200 registers).
+// Tensor memory (fp32 columns x 128 lanes):
+//   D = 128 (T = 2, 512 columns): S_t = Q_t K_j^T at [128 t, 128 t + 128), P_t
+//     (16-bit, two per column) aliasing the first 64 columns of S_t, O_t += P_t V_j
+//     at [256 + 128 t, ...).  One issuer runs PV_0(j), QK_0(j+1), PV_1(j),
+//     QK_1(j+1); each commit to S_t's barrier also covers the PV_t(j) issued before
+//     it, so when a softmax warpgroup sees S_t(j+1) it knows P_t(j) has been
+//     consumed and O_t is up to date; it may then rescale O_t before releasing
+//     P_t(j+1).
+//   D = 64 (256 T columns): S_t at [128 t, ...), P_t at [128 T + 64 t, ...), O_t at
+//     [192 T + 64 t, ...).  Each tile has its own issuer, and QK_t(j+1) is issued as
+//     soon as S_t(j) sits in registers.
 // The running max is kept lazily: O is rescaled only when a row's max grows by
 // more than 8 (base-2 units); the final O / l and LSE use the same stale max, so
 // the result is unchanged.  Blocks that lie fully inside every row's allowed key
@@ -43,22 +43,33 @@ namespace fa {
 
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per K/V block
-constexpr int kFwdThreads = 384;
-// 2*128*200 + 128*104 = 64512 = 384*168 (the registers the CTA launches with)
 constexpr uint32_t kSoftmaxRegs = 200;
-constexpr uint32_t kOtherRegs = 104;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
-template <int D>
+// T query tiles per CTA (1 or 2).  With T = 2 one CTA fills an SM (512 TMEM
+// columns, 12 warps); with T = 1 two CTAs share an SM (256 columns and 8 warps
+// each) and, being independent, drift out of phase, so that one CTA's
+// exponentials overlap the other's loads and reductions.
+template <int D, int T>
 struct FwdCfg {
+  static_assert(T == 1 || T == 2, "one or two query tiles per CTA");
+  static_assert(T == 2 || D == 64, "one tile per CTA is laid out for D = 64 only");
+  static constexpr int kThreads = (4 * T + 4) * 32;   // softmax warpgroups + one more
+  static constexpr int kMinBlocks = 3 - T;             // CTAs per SM
+  // registers a thread launches with, and what the non-softmax warpgroup keeps:
+  // T*128*200 + 128*kOtherRegs = kThreads * kLaunchRegs
+  static constexpr int kLaunchRegs = (T == 2) ? 168 : 128;
+  static constexpr uint32_t kOtherRegs = (T == 2) ? 104 : 56;
+  static_assert(T * 128 * kSoftmaxRegs + 128 * kOtherRegs == kThreads * kLaunchRegs,
+                "register re-split must add up to the launch registers");
   static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms per row
-  static constexpr int kStages = (D == 128) ? 2 : 4;  // K and V ring depth
+  static constexpr int kStages = (D == 128) ? 2 : (T == 2 ? 4 : 2);  // K and V ring depth
   static constexpr int kTileBytes = 128 * D * 2;      // Q tile, K block or V block
   static constexpr int kChunkBytes = 128 * 128;       // 128 rows x 128 bytes
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + 2 * kTileBytes;
+  static constexpr int kKOff = kQOff + T * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
@@ -67,14 +78,17 @@ struct FwdCfg {
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // room to align the base to 1 KiB
-  static constexpr int kTmemCols = 512;
-  // D = 64: P has its own columns (S 2x128, P 2x64, O 2x64 = 512), so the next
-  // S can be computed while the softmax still works on the current one.
+  static constexpr int kTmemCols = 256 * T;
+  // D = 64: P has its own columns (S Tx128, P Tx64, O Tx64), so the next S can be
+  // computed while the softmax still works on the current one.
   // D = 128: S 2x128 + O 2x128 fill the 512 columns and P aliases S.
   static constexpr bool kSepP = (D == 64);
-  static constexpr int kPCol = kSepP ? 256 : 0;
+  static constexpr int kPCol = kSepP ? 128 * T : 0;
   static constexpr int kPStride = kSepP ? 64 : 128;
-  static constexpr int kOCol = kSepP ? 384 : 256;
+  static constexpr int kOCol = kSepP ? 192 * T : 256;
+  // warp roles: 4T softmax warps, then the producer, then the MMA issuer(s)
+  static constexpr int kProducerWarp = 4 * T;
+  static constexpr int kIssuerWarp = 4 * T + 1;  // also allocates tensor memory
 };
 
 // Wait that ignores the abort flag (used to drain this CTA's own in-flight work).
@@ -112,11 +126,11 @@ __device__ __forceinline__ void fwd_issue_pv(uint32_t d_tmem, uint32_t a_tmem, u
            (acc || kk > 0) ? 1u : 0u);
 }
 
-template <int D, bool BF16, bool SOFTCAP, bool ALIBI, int EMU>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+template <int D, int T, bool BF16, bool SOFTCAP, bool ALIBI, int EMU>
+__global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBlocks)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using Cfg = FwdCfg<D>;
+  using Cfg = FwdCfg<D, T>;
   constexpr int ST = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -136,10 +150,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     k0 = p.cu_k[b];
     Sk_b = p.cu_k[b + 1] - k0;
   }
-  const int n_pairs_b = (Sq_b + 2 * kBM - 1) / (2 * kBM);
-  if (static_cast<int>(blockIdx.z) >= n_pairs_b) return;  // uniform: whole CTA leaves
-  const int pair = n_pairs_b - 1 - static_cast<int>(blockIdx.z);  // heaviest rows first
-  const int row0 = pair * 2 * kBM;
+  const int n_units_b = (Sq_b + T * kBM - 1) / (T * kBM);
+  if (static_cast<int>(blockIdx.z) >= n_units_b) return;  // uniform: whole CTA leaves
+  const int unit = n_units_b - 1 - static_cast<int>(blockIdx.z);  // heaviest rows first
+  const int row0 = unit * T * kBM;
   const int off = Sk_b - Sq_b;  // bottom-right alignment
   const bool has_left = p.wl >= 0;
   const bool has_right = p.causal || p.wr >= 0;
@@ -147,7 +161,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // allowed keys of row i: [lo(i), hi(i)] intersected with [0, Sk_b)
   auto lo_of = [&](int i) { return has_left ? i + off - p.wl : INT_MIN / 2; };
   auto hi_of = [&](int i) { return has_right ? min(i + off + right, Sk_b - 1) : Sk_b - 1; };
-  const int r_last = min(row0 + 2 * kBM - 1, Sq_b - 1);
+  const int r_last = min(row0 + T * kBM - 1, Sq_b - 1);
   const int k_begin = max(0, lo_of(row0));
   const int k_end = hi_of(r_last) + 1;  // exclusive
   const int j_lo = k_begin / kBN;
@@ -172,13 +186,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
-  if (warp == 8 && lane == 0) {
+  if (warp == Cfg::kProducerWarp && lane == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < ST; ++s) {
       mbar_init(k_full + s, 1);
-      mbar_init(k_empty + s, 2);  // released by both issuers
+      mbar_init(k_empty + s, T);  // released once per tile
       mbar_init(v_full + s, 1);
-      mbar_init(v_empty + s, 2);
+      mbar_init(v_empty + s, T);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full + t, 1);
@@ -192,7 +206,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == Cfg::kIssuerWarp) {
     tmem_alloc(tmem_holder, Cfg::kTmemCols);
     tmem_relinquish();
   }
@@ -203,9 +217,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const WaitCtx w{abort_flag, p.status, p.timeout_ns};
   const bool varlen = p.cu_q != nullptr;
   const int b_coord = varlen ? 0 : b;
-  if (warp >= 8) {
-   regs_dec<kOtherRegs>();
-   if (warp == 8) {
+  if (warp >= Cfg::kProducerWarp) {
+   regs_dec<Cfg::kOtherRegs>();
+   if (warp == Cfg::kProducerWarp) {
     // ======================================================== TMA producer
     if (lane == 0 && n_blk > 0) {
       tma_prefetch_map(&tmQ);
@@ -213,8 +227,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tma_prefetch_map(&tmV);
       const int qrow = (varlen ? q0 : 0) + row0;
       const int krow = varlen ? k0 : 0;
-      mbar_arrive_expect_tx(q_full, 2 * Cfg::kTileBytes);
-      for (int t = 0; t < 2; ++t)
+      mbar_arrive_expect_tx(q_full, T * Cfg::kTileBytes);
+      for (int t = 0; t < T; ++t)
         for (int c = 0; c < Cfg::kChunks; ++c)
           tma_load_4d(sQ + t * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmQ, q_full, c * 64,
                       qrow + t * kBM, h, b_coord);
@@ -246,7 +260,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
     __syncwarp();
-   } else if (warp == 9 && !Cfg::kSepP) {
+   } else if (warp == Cfg::kIssuerWarp && !Cfg::kSepP) {
     // ======================================================== MMA issuer (D = 128)
     // One thread alternates the tiles, PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so
     // one tile's softmax overlaps the other tile's products.
@@ -311,9 +325,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       wait_drain(drain + 0, 0, p.timeout_ns);
     }
     __syncwarp();
-   } else if (Cfg::kSepP && (warp == 9 || warp == 10)) {
+   } else if (Cfg::kSepP && warp >= Cfg::kIssuerWarp && warp < Cfg::kIssuerWarp + T) {
     // ======================================================== MMA issuers (D = 64)
-    const int t = warp - 9;  // this issuer's query tile
+    const int t = warp - Cfg::kIssuerWarp;  // this issuer's query tile
     if (lane == 0 && n_blk > 0) {
       constexpr uint32_t idesc_qk = f16_idesc(BF16, kBM, kBN, false, false);
       constexpr uint32_t idesc_pv = f16_idesc(BF16, kBM, D, false, true);
@@ -606,7 +620,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // ---------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == Cfg::kIssuerWarp) {
     tc_fence_after();
     tmem_dealloc(tbase, Cfg::kTmemCols);
   }

@@ -8,16 +8,21 @@
 
 namespace fa {
 
-template <int D, bool BF16, bool SOFTCAP, bool ALIBI, int EMU>
+template <int D, int T, bool BF16, bool SOFTCAP, bool ALIBI, int EMU>
 cudaError_t launch_fwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const FwdParams& p, int batch, int n_pairs, cudaStream_t stream) {
-  auto kern = fwd_kernel<D, BF16, SOFTCAP, ALIBI, EMU>;
-  constexpr int smem = FwdCfg<D>::kSmemAlloc;
+                            const FwdParams& p, int batch, int rows_q, cudaStream_t stream) {
+  using Cfg = FwdCfg<D, T>;
+  auto kern = fwd_kernel<D, T, BF16, SOFTCAP, ALIBI, EMU>;
+  constexpr int smem = Cfg::kSmemAlloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess && T == 1)  // room for two CTAs per SM
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
+  const int n_units = (rows_q + T * kBM - 1) / (T * kBM);
   const dim3 grid(static_cast<unsigned>(p.H), static_cast<unsigned>(batch),
-                  static_cast<unsigned>(n_pairs));
-  kern<<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, p);
+                  static_cast<unsigned>(n_units));
+  kern<<<grid, Cfg::kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -32,30 +37,49 @@ inline int exp2_emu_choice(int d) {
   return d == 64 ? 2 : 0;
 }
 
+// Query tiles per CTA at D = 64 (D = 128 always takes two); FA_FWD_TILES in the
+// environment overrides (1 or 2).
+inline int fwd_tiles_choice() {
+  static const int env = [] {
+    const char* e = std::getenv("FA_FWD_TILES");
+    return e ? std::atoi(e) : -1;
+  }();
+  if (env == 1 || env == 2) return env;
+  return 2;
+}
+
 template <bool BF16>
 cudaError_t launch_fwd_dtype(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const FwdParams& p, int d, int batch, int n_pairs,
+                             const FwdParams& p, int d, int batch, int rows_q,
                              cudaStream_t stream) {
   const bool sc = p.softcap_log2 > 0.f;
   const bool al = p.alibi != nullptr;
   const int emu = (sc || al) ? 0 : exp2_emu_choice(d);
-#define FA_FWD_CASE(DD, SC, AL, EM)                                                        \
-  if (d == DD && sc == SC && al == AL && emu == EM)                                        \
-    return launch_fwd_inst<DD, BF16, SC, AL, EM>(tq, tk, tv, p, batch, n_pairs, stream);
-  FA_FWD_CASE(64, false, false, 0)
-  FA_FWD_CASE(64, false, false, 2)
-  FA_FWD_CASE(64, false, false, 3)
-  FA_FWD_CASE(64, false, false, 4)
-  FA_FWD_CASE(64, true, false, 0)
-  FA_FWD_CASE(64, false, true, 0)
-  FA_FWD_CASE(64, true, true, 0)
-  FA_FWD_CASE(128, false, false, 0)
-  FA_FWD_CASE(128, false, false, 2)
-  FA_FWD_CASE(128, false, false, 3)
-  FA_FWD_CASE(128, false, false, 4)
-  FA_FWD_CASE(128, true, false, 0)
-  FA_FWD_CASE(128, false, true, 0)
-  FA_FWD_CASE(128, true, true, 0)
+  const int tiles = (d == 64) ? fwd_tiles_choice() : 2;
+#define FA_FWD_CASE(DD, TT, SC, AL, EM)                                                    \
+  if (d == DD && tiles == TT && sc == SC && al == AL && emu == EM)                         \
+    return launch_fwd_inst<DD, TT, BF16, SC, AL, EM>(tq, tk, tv, p, batch, rows_q, stream);
+  FA_FWD_CASE(64, 1, false, false, 0)
+  FA_FWD_CASE(64, 1, false, false, 2)
+  FA_FWD_CASE(64, 1, false, false, 3)
+  FA_FWD_CASE(64, 1, false, false, 4)
+  FA_FWD_CASE(64, 1, true, false, 0)
+  FA_FWD_CASE(64, 1, false, true, 0)
+  FA_FWD_CASE(64, 1, true, true, 0)
+  FA_FWD_CASE(64, 2, false, false, 0)
+  FA_FWD_CASE(64, 2, false, false, 2)
+  FA_FWD_CASE(64, 2, false, false, 3)
+  FA_FWD_CASE(64, 2, false, false, 4)
+  FA_FWD_CASE(64, 2, true, false, 0)
+  FA_FWD_CASE(64, 2, false, true, 0)
+  FA_FWD_CASE(64, 2, true, true, 0)
+  FA_FWD_CASE(128, 2, false, false, 0)
+  FA_FWD_CASE(128, 2, false, false, 2)
+  FA_FWD_CASE(128, 2, false, false, 3)
+  FA_FWD_CASE(128, 2, false, false, 4)
+  FA_FWD_CASE(128, 2, true, false, 0)
+  FA_FWD_CASE(128, 2, false, true, 0)
+  FA_FWD_CASE(128, 2, true, true, 0)
 #undef FA_FWD_CASE
   return cudaErrorInvalidValue;
 }
