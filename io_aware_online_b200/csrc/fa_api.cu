@@ -294,6 +294,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
   p.causal = causal ? 1 : 0;
   p.wl = window_left;
   p.wr = window_right;
+  p.tile_major = (!causal && window_left < 0 && window_right < 0) ? 1 : 0;
   p.status = status;
   p.timeout_ns = timeout_ns();
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -23,6 +23,7 @@ struct FwdParams {
   float tanh_k;                    // 2 * log2(e) * softmax_scale / softcap
   const float* alibi;              // [H] or NULL
   int causal, wl, wr;              // mask flags; -1 = unbounded window side
+  int tile_major;                  // grid x = query tiles (no mask: equal work per tile)
   unsigned int* status;            // device status word
   uint64_t timeout_ns;             // bounded-wait limit
 };

@@ -138,8 +138,12 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int h = blockIdx.x;
-  const int b = blockIdx.y;
+  // grid order: query tiles fastest when every tile does the same work (the
+  // tiles of a head then run together and share its K/V in L2), else heads
+  // fastest with the heaviest tiles first (balance under a causal or window mask)
+  const int h = p.tile_major ? blockIdx.y : blockIdx.x;
+  const int b = p.tile_major ? blockIdx.z : blockIdx.y;
+  const int zi = static_cast<int>(p.tile_major ? blockIdx.x : blockIdx.z);
   const int hk = h / p.G;
 
   // ---------------------------------------------------------- problem geometry
@@ -151,8 +155,8 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
     Sk_b = p.cu_k[b + 1] - k0;
   }
   const int n_units_b = (Sq_b + T * kBM - 1) / (T * kBM);
-  if (static_cast<int>(blockIdx.z) >= n_units_b) return;  // uniform: whole CTA leaves
-  const int unit = n_units_b - 1 - static_cast<int>(blockIdx.z);  // heaviest rows first
+  if (zi >= n_units_b) return;  // uniform: whole CTA leaves
+  const int unit = n_units_b - 1 - zi;  // heaviest rows first
   const int row0 = unit * T * kBM;
   const int off = Sk_b - Sq_b;  // bottom-right alignment
   const bool has_left = p.wl >= 0;

@@ -20,8 +20,10 @@ cudaError_t launch_fwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const 
                              cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   const int n_units = (rows_q + T * kBM - 1) / (T * kBM);
-  const dim3 grid(static_cast<unsigned>(p.H), static_cast<unsigned>(batch),
-                  static_cast<unsigned>(n_units));
+  const dim3 grid = p.tile_major ? dim3(static_cast<unsigned>(n_units), static_cast<unsigned>(p.H),
+                                         static_cast<unsigned>(batch))
+                                  : dim3(static_cast<unsigned>(p.H), static_cast<unsigned>(batch),
+                                         static_cast<unsigned>(n_units));
   kern<<<grid, Cfg::kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
