@@ -69,7 +69,11 @@ enum fa_dtype { FA_FP16 = 0, FA_BF16 = 1, FA_FP32 = 2 /* fa_combine output only 
 /* Device status bits (fa_device_status). */
 enum fa_device_flag {
     FA_DEV_WAIT_TIMEOUT = 1u,   /* a pipeline wait exceeded its time limit; that CTA stopped */
-    FA_DEV_BAD_BLOCK = 2u       /* a block_table entry was outside [0, num_blocks) */
+    FA_DEV_BAD_BLOCK = 2u,      /* a block_table entry was outside [0, num_blocks) */
+    FA_DEV_BAD_LENGTH = 4u      /* a cache length (cache_seqlens[b], plus appended keys)
+                                   was negative or beyond the cache's capacity; the
+                                   kernel clamped it (attention) or skipped the row
+                                   (append) */
 };
 
 /*
@@ -122,7 +126,8 @@ FA_API size_t fa_kvcache_workspace_size(int batch, int seqlen_q, int num_heads, 
 /*
  * fa_fwd_kvcache -- attention of a few new query rows against a KV cache,
  * split along the keys (changelog v2.2 split-KV "flash-decoding"; v2.5 paged KV
- * cache; section 3.3 flash_attn_with_kvcache without the in-place append).
+ * cache; section 3.3 flash_attn_with_kvcache; the in-place append of new keys is
+ * fa_fwd_kvcache_append).
  *
  *   q   [batch, seqlen_q, num_heads, head_dim] contiguous; out like q;
  *   lse fp32 [batch, num_heads, seqlen_q] or NULL.
@@ -156,6 +161,53 @@ FA_API int fa_fwd_kvcache(const void *q, const void *k_cache, const void *v_cach
                    int window_left, int window_right, float softcap,
                    const float *alibi_slopes, int num_splits, void *workspace,
                    size_t workspace_bytes, void *stream);
+
+/*
+ * fa_kvcache_append -- write new keys and values into a KV cache in place, at the
+ * positions after each sequence's cached keys (section 3.3: flash_attn_with_kvcache
+ * with k and v given "updates the cache").
+ *
+ *   k_new, v_new [batch, seqlen_new, num_heads_k, head_dim] contiguous, 16-bit
+ *   (dtype as for fa_fwd).  Row t of sequence b goes to key position
+ *   cache_seqlens[b] + t of that sequence: cache_seqlens is the number of keys
+ *   ALREADY in the cache, before this append (the parameter's description on
+ *   the page; its worked example's 128-then-129 values read as lengths after the
+ *   append and are not followed).  cache_seqlens is required and is not updated:
+ *   the caller advances it by seqlen_new for the next step.
+ * Paged cache (block_table != NULL): position x of sequence b is row x % page_size
+ *   of pool block block_table[b, x / page_size]; the cache layout and arguments are
+ *   those of fa_fwd_kvcache.  Contiguous cache (block_table == NULL): row x of
+ *   sequence b of k_cache [batch, seqlen_k_max, num_heads_k, head_dim].
+ * A position outside the cache's capacity (max_blocks_per_seq * page_size or
+ *   seqlen_k_max) or a block_table entry outside [0, num_blocks) is not written;
+ *   the kernel raises FA_DEV_BAD_LENGTH or FA_DEV_BAD_BLOCK (fa_device_status).
+ * Writes nothing else.  Asynchronous on `stream`; allocates nothing.
+ */
+FA_API int fa_kvcache_append(void *k_cache, void *v_cache, const void *k_new, const void *v_new,
+                             int dtype, int batch, int seqlen_new, int num_heads_k, int head_dim,
+                             const int32_t *block_table, int max_blocks_per_seq, int page_size,
+                             int num_blocks, int seqlen_k_max, const int32_t *cache_seqlens,
+                             void *stream);
+
+/*
+ * fa_fwd_kvcache_append -- fa_kvcache_append followed, on the same stream, by
+ * fa_fwd_kvcache over the grown cache (section 3.3 with k and v given): sequence
+ * b then attends its cache_seqlens[b] + seqlen_new keys, and with causal the
+ * query rows sit at the last seqlen_q of those positions (bottom-right).  The
+ * arguments are those of fa_fwd_kvcache (cache_seqlens still counts the keys
+ * before the append and is required) plus k_new, v_new and seqlen_new as for
+ * fa_kvcache_append; the workspace rule is fa_fwd_kvcache's.
+ */
+FA_API int fa_fwd_kvcache_append(const void *q, void *k_cache, void *v_cache, const void *k_new,
+                                 const void *v_new, int seqlen_new, void *out, float *lse,
+                                 int dtype, int batch, int seqlen_q, int num_heads,
+                                 int num_heads_k, int head_dim, const int32_t *block_table,
+                                 int max_blocks_per_seq, int page_size, int num_blocks,
+                                 int seqlen_k_max, const int32_t *cache_seqlens,
+                                 float softmax_scale, int causal, int window_left,
+                                 int window_right, float softcap, const float *alibi_slopes,
+                                 int num_splits, void *workspace, size_t workspace_bytes,
+                                 void *stream);
 
 /*
  * fa_fwd_kvcache_static -- fa_fwd_kvcache without a workspace argument, for callers

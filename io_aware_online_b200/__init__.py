@@ -70,6 +70,13 @@ def load():
                                           i32, i32, i32, i32, vp, f32, i32, i32, i32, f32, vp,
                                           i32, vp]
     lib.fa_fwd_kvcache_static.restype = i32
+    lib.fa_kvcache_append.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, i32, i32, i32,
+                                      i32, vp, vp]
+    lib.fa_kvcache_append.restype = i32
+    lib.fa_fwd_kvcache_append.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
+                                          i32, i32, vp, i32, i32, i32, i32, vp, f32, i32, i32,
+                                          i32, f32, vp, i32, vp, ctypes.c_size_t, vp]
+    lib.fa_fwd_kvcache_append.restype = i32
     lib.fa_kvcache_static_scratch_bytes.argtypes = []
     lib.fa_kvcache_static_scratch_bytes.restype = ctypes.c_size_t
     lib.fa_combine.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64p, i64p, vp]
@@ -192,20 +199,47 @@ def fa_kvcache_workspace_size(batch, seqlen_q, num_heads, num_heads_k, head_dim,
                                                 head_dim, max_seqlen_k, page_size, num_splits))
 
 
-def fa_fwd_kvcache(q, k_cache, v_cache, *, cache_seqlens=None, block_table=None,
+def _cache_geometry(k_cache, block_table):
+    if block_table is not None:
+        return k_cache.shape[2], k_cache.shape[0], k_cache.shape[1], block_table.shape[1], 0
+    return k_cache.shape[2], 0, 0, 0, k_cache.shape[1]   # Hkv, num_blocks, page, max_blocks, sk_max
+
+
+def fa_kvcache_append(k_cache, v_cache, k, v, cache_seqlens, *, block_table=None, stream=None):
+    """Write k, v [B, S_new, Hkv, d] into the cache at positions cache_seqlens[b] + t
+    (cache_seqlens = keys already cached; it is not advanced here)."""
+    lib = load()
+    dt = _dtype(k)
+    B, s_new, Hkv, d = k.shape
+    for t in (k_cache, v_cache, k, v):
+        if not t.is_contiguous():
+            raise ValueError("the caches and the new keys/values must be contiguous")
+    _, num_blocks, page, max_blocks, sk_max = _cache_geometry(k_cache, block_table)
+    _check(lib.fa_kvcache_append(_ptr(k_cache), _ptr(v_cache), _ptr(k), _ptr(v), dt, B, s_new,
+                                 Hkv, d, _ptr(block_table), max_blocks, page, num_blocks, sk_max,
+                                 _ptr(cache_seqlens), _stream(stream)))
+
+
+def fa_fwd_kvcache(q, k_cache, v_cache, k=None, v=None, *, cache_seqlens=None, block_table=None,
                    softmax_scale=None, causal=False, window_size=(-1, -1), softcap=0.0,
                    alibi_slopes=None, num_splits=0, out=None, lse=None, return_lse=True,
                    workspace=None, stream=None):
-    """Split-KV attention against a paged or contiguous KV cache (section 3.3,
-    without the in-place append).  q [B, Sq, H, d]; paged pools
-    [num_blocks, page, Hkv, d] with int32 block_table [B, max_blocks]; or
-    contiguous caches [B, Sk_max, Hkv, d]."""
+    """Split-KV attention against a paged or contiguous KV cache (section 3.3).
+    q [B, Sq, H, d]; paged pools [num_blocks, page, Hkv, d] with int32 block_table
+    [B, max_blocks]; or contiguous caches [B, Sk_max, Hkv, d].  With k and v
+    [B, S_new, Hkv, d] given, they are first written into the cache after the
+    cache_seqlens[b] keys already there, and the attention covers
+    cache_seqlens[b] + S_new keys (cache_seqlens itself is not advanced)."""
     lib = load()
     dt = _dtype(q)
     B, sq, H, d = q.shape
     for t in (q, k_cache, v_cache):
         if not t.is_contiguous():
             raise ValueError("q and the caches must be contiguous")
+    if (k is None) != (v is None):
+        raise ValueError("give both k and v, or neither")
+    if k is not None and not (k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("k and v must be contiguous")
     if block_table is not None:
         num_blocks, page, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
         max_blocks = block_table.shape[1]
@@ -223,12 +257,22 @@ def fa_fwd_kvcache(q, k_cache, v_cache, *, cache_seqlens=None, block_table=None,
         out = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, H, sq), dtype=torch.float32, device=q.device)
-    _check(lib.fa_fwd_kvcache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), dt,
-                              B, sq, H, Hkv, d, _ptr(block_table), max_blocks, page, num_blocks,
-                              sk_max, _ptr(cache_seqlens), _scale(softmax_scale),
-                              int(bool(causal)), int(window_size[0]), int(window_size[1]),
-                              float(softcap), _ptr(alibi_slopes), int(num_splits),
-                              _ptr(workspace), ws_bytes, _stream(stream)))
+    if k is None:
+        _check(lib.fa_fwd_kvcache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
+                                  dt, B, sq, H, Hkv, d, _ptr(block_table), max_blocks, page,
+                                  num_blocks, sk_max, _ptr(cache_seqlens), _scale(softmax_scale),
+                                  int(bool(causal)), int(window_size[0]), int(window_size[1]),
+                                  float(softcap), _ptr(alibi_slopes), int(num_splits),
+                                  _ptr(workspace), ws_bytes, _stream(stream)))
+    else:
+        _check(lib.fa_fwd_kvcache_append(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k), _ptr(v),
+                                         k.shape[1], _ptr(out), _ptr(lse), dt, B, sq, H, Hkv, d,
+                                         _ptr(block_table), max_blocks, page, num_blocks, sk_max,
+                                         _ptr(cache_seqlens), _scale(softmax_scale),
+                                         int(bool(causal)), int(window_size[0]),
+                                         int(window_size[1]), float(softcap),
+                                         _ptr(alibi_slopes), int(num_splits), _ptr(workspace),
+                                         ws_bytes, _stream(stream)))
     return out, lse
 
 

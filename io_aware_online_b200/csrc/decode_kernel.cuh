@@ -105,7 +105,16 @@ __device__ __forceinline__ DecItem dec_item(const DecodeParams& p, int item) {
   it.split = item % p.num_splits;
   it.hk = (item / p.num_splits) % p.Hkv;
   it.b = item / (p.num_splits * p.Hkv);
-  it.L = (p.cache_seqlens != nullptr) ? p.cache_seqlens[it.b] : p.seqlen_k_max;
+  it.L = ((p.cache_seqlens != nullptr) ? p.cache_seqlens[it.b] : p.seqlen_k_max) + p.k_add;
+  {
+    // a length the cache cannot hold would read past the block table: clamp it
+    // and report (identically in the producer and the consumers)
+    const int cap = (p.block_table != nullptr) ? p.max_blocks * p.page_size : p.seqlen_k_max;
+    if (it.L < 0 || it.L > cap) {
+      atomicOr(p.status, kDevBadLength);
+      it.L = min(max(it.L, 0), cap);
+    }
+  }
   const int n_units = (it.L + p.unit - 1) / p.unit;
   const int per = (n_units + p.num_splits - 1) / p.num_splits;
   const int u_begin = it.split * per;

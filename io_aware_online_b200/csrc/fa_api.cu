@@ -327,18 +327,19 @@ size_t fa_kvcache_workspace_size(int batch, int seqlen_q, int num_heads, int num
          static_cast<size_t>(s) * batch * seqlen_q * num_heads * (head_dim + 1) * sizeof(float);
 }
 
-int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void* out, float* lse,
-                   int dtype, int batch, int seqlen_q, int num_heads, int num_heads_k,
-                   int head_dim, const int32_t* block_table, int max_blocks_per_seq,
-                   int page_size, int num_blocks, int seqlen_k_max,
-                   const int32_t* cache_seqlens, float softmax_scale, int causal,
-                   int window_left, int window_right, float softcap,
-                   const float* alibi_slopes, int num_splits, void* workspace,
-                   size_t workspace_bytes, void* stream) {
-  g_err.clear();
+// fa_fwd_kvcache's body.  `app` (optional) is an append of k_add new keys per
+// sequence, launched on the same stream once every argument has been checked.
+static int kvcache_impl(const void* q, const void* k_cache, const void* v_cache, void* out,
+                        float* lse, int dtype, int batch, int seqlen_q, int num_heads,
+                        int num_heads_k, int head_dim, const int32_t* block_table,
+                        int max_blocks_per_seq, int page_size, int num_blocks, int seqlen_k_max,
+                        const int32_t* cache_seqlens, float softmax_scale, int causal,
+                        int window_left, int window_right, float softcap,
+                        const float* alibi_slopes, int num_splits, void* workspace,
+                        size_t workspace_bytes, void* stream, fa::AppendParams* app) {
   int rc = check_common(dtype, head_dim, num_heads, num_heads_k, window_left, window_right, softcap);
   if (rc != FA_OK) return rc;
-  if (!q || !k_cache || !v_cache || !out)
+  if (!k_cache || !v_cache || ((!q || !out) && batch > 0 && seqlen_q > 0))
     return fail(FA_ERR_INVALID_ARG, "fa_fwd_kvcache: q, k_cache, v_cache and out must be non-NULL");
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
     return fail(FA_ERR_INVALID_ARG, "fa_fwd_kvcache: q, caches and out must be 16-byte aligned");
@@ -366,9 +367,17 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
   }
   float scale;
   if ((rc = resolve_scale(softmax_scale, d, &scale)) != FA_OK) return rc;
-  if (batch == 0 || seqlen_q == 0) return FA_OK;
   if (batch > 65535 || Hkv > 65535)
     return fail(FA_ERR_UNSUPPORTED, "fa_fwd_kvcache: batch or num_heads_k above 65535");
+  if (batch == 0) return FA_OK;
+  if (seqlen_q == 0) {  // nothing to attend; an append still happens
+    if (app == nullptr) return FA_OK;
+    unsigned int* st0 = nullptr;
+    if ((rc = device_state(nullptr, &st0, nullptr)) != FA_OK) return rc;
+    app->status = st0;
+    const cudaError_t e0 = fa::launch_kv_append(*app, static_cast<cudaStream_t>(stream));
+    return e0 == cudaSuccess ? FA_OK : cuda_fail(e0, "fa_fwd_kvcache_append append launch");
+  }
   const int splits = resolve_splits(batch, seqlen_q, H, Hkv, d, max_k, unit, num_splits);
   const size_t need = fa_kvcache_workspace_size(batch, seqlen_q, H, Hkv, d, max_k,
                                                 paged ? page_size : 0, num_splits);
@@ -410,6 +419,7 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
   p.item_counter = static_cast<unsigned int*>(workspace);
   p.block_table = block_table;
   p.cache_seqlens = cache_seqlens;
+  p.k_add = app ? app->S_new : 0;
   p.B = batch;
   p.Sq = seqlen_q;
   p.H = H;
@@ -432,7 +442,13 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
   p.timeout_ns = timeout_ns();
   p.sm_count = sms;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(p.item_counter, 0, sizeof(unsigned int), s);
+  cudaError_t e;
+  if (app != nullptr) {
+    app->status = status;
+    e = fa::launch_kv_append(*app, s);
+    if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache_append append launch");
+  }
+  e = cudaMemsetAsync(p.item_counter, 0, sizeof(unsigned int), s);
   if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache counter reset");
   e = fa::launch_decode(tk, tv, p, dtype == FA_BF16, d, s);
   if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache split kernel launch");
@@ -462,6 +478,102 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
     if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache combine launch");
   }
   return FA_OK;
+}
+
+int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void* out, float* lse,
+                   int dtype, int batch, int seqlen_q, int num_heads, int num_heads_k,
+                   int head_dim, const int32_t* block_table, int max_blocks_per_seq,
+                   int page_size, int num_blocks, int seqlen_k_max,
+                   const int32_t* cache_seqlens, float softmax_scale, int causal,
+                   int window_left, int window_right, float softcap,
+                   const float* alibi_slopes, int num_splits, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  return kvcache_impl(q, k_cache, v_cache, out, lse, dtype, batch, seqlen_q, num_heads,
+                      num_heads_k, head_dim, block_table, max_blocks_per_seq, page_size,
+                      num_blocks, seqlen_k_max, cache_seqlens, softmax_scale, causal, window_left,
+                      window_right, softcap, alibi_slopes, num_splits, workspace, workspace_bytes,
+                      stream, nullptr);
+}
+
+// Checks the arguments of an append and fills `a` (status left for the caller).
+static int append_args(void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                       int dtype, int batch, int seqlen_new, int num_heads_k, int head_dim,
+                       const int32_t* block_table, int max_blocks_per_seq, int page_size,
+                       int num_blocks, int seqlen_k_max, const int32_t* cache_seqlens,
+                       fa::AppendParams* a) {
+  if (dtype != FA_FP16 && dtype != FA_BF16)
+    return fail(FA_ERR_UNSUPPORTED, "kv append: dtype must be FA_FP16 or FA_BF16");
+  if (head_dim <= 0 || head_dim > 256 || head_dim % 8)
+    return fail(FA_ERR_UNSUPPORTED, "kv append: head_dim %d (a multiple of 8 up to 256)", head_dim);
+  if (batch < 0 || seqlen_new < 0 || num_heads_k <= 0)
+    return fail(FA_ERR_INVALID_ARG, "kv append: negative size or num_heads_k <= 0");
+  if (!k_cache || !v_cache || (seqlen_new > 0 && batch > 0 && (!k_new || !v_new)))
+    return fail(FA_ERR_INVALID_ARG, "kv append: caches and new keys/values must be non-NULL");
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) || !aligned16(v_new))
+    return fail(FA_ERR_INVALID_ARG, "kv append: caches and new keys/values must be 16-byte aligned");
+  if (cache_seqlens == nullptr)
+    return fail(FA_ERR_INVALID_ARG, "kv append: cache_seqlens (keys before the append) is required");
+  if (block_table != nullptr) {
+    if (page_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+      return fail(FA_ERR_INVALID_ARG, "kv append: page_size, num_blocks and max_blocks_per_seq must be positive");
+  } else if (seqlen_k_max < 0) {
+    return fail(FA_ERR_INVALID_ARG, "kv append: seqlen_k_max < 0");
+  }
+  *a = fa::AppendParams{};
+  a->k_cache = k_cache;
+  a->v_cache = v_cache;
+  a->k_new = k_new;
+  a->v_new = v_new;
+  a->block_table = block_table;
+  a->cache_seqlens = cache_seqlens;
+  a->B = batch;
+  a->S_new = seqlen_new;
+  a->Hkv = num_heads_k;
+  a->D = head_dim;
+  a->max_blocks = max_blocks_per_seq;
+  a->page_size = page_size;
+  a->num_blocks = num_blocks;
+  a->seqlen_k_max = seqlen_k_max;
+  return FA_OK;
+}
+
+int fa_kvcache_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                      int dtype, int batch, int seqlen_new, int num_heads_k, int head_dim,
+                      const int32_t* block_table, int max_blocks_per_seq, int page_size,
+                      int num_blocks, int seqlen_k_max, const int32_t* cache_seqlens,
+                      void* stream) {
+  g_err.clear();
+  fa::AppendParams a;
+  int rc = append_args(k_cache, v_cache, k_new, v_new, dtype, batch, seqlen_new, num_heads_k,
+                       head_dim, block_table, max_blocks_per_seq, page_size, num_blocks,
+                       seqlen_k_max, cache_seqlens, &a);
+  if (rc != FA_OK) return rc;
+  if (batch == 0 || seqlen_new == 0) return FA_OK;
+  if ((rc = device_state(nullptr, &a.status, nullptr)) != FA_OK) return rc;
+  const cudaError_t e = fa::launch_kv_append(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e, "fa_kvcache_append launch");
+}
+
+int fa_fwd_kvcache_append(const void* q, void* k_cache, void* v_cache, const void* k_new,
+                          const void* v_new, int seqlen_new, void* out, float* lse, int dtype,
+                          int batch, int seqlen_q, int num_heads, int num_heads_k, int head_dim,
+                          const int32_t* block_table, int max_blocks_per_seq, int page_size,
+                          int num_blocks, int seqlen_k_max, const int32_t* cache_seqlens,
+                          float softmax_scale, int causal, int window_left, int window_right,
+                          float softcap, const float* alibi_slopes, int num_splits,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  fa::AppendParams a;
+  int rc = append_args(k_cache, v_cache, k_new, v_new, dtype, batch, seqlen_new, num_heads_k,
+                       head_dim, block_table, max_blocks_per_seq, page_size, num_blocks,
+                       seqlen_k_max, cache_seqlens, &a);
+  if (rc != FA_OK) return rc;
+  return kvcache_impl(q, k_cache, v_cache, out, lse, dtype, batch, seqlen_q, num_heads,
+                      num_heads_k, head_dim, block_table, max_blocks_per_seq, page_size,
+                      num_blocks, seqlen_k_max, cache_seqlens, softmax_scale, causal, window_left,
+                      window_right, softcap, alibi_slopes, num_splits, workspace, workspace_bytes,
+                      stream, seqlen_new > 0 ? &a : nullptr);
 }
 
 int fa_combine(const float* out_partial, const float* lse_partial, void* out, float* lse,

@@ -37,6 +37,7 @@ struct DecodeParams {
   float* ws_lse;                   // [splits, B, Sq, H]
   const int32_t* block_table;      // [B, max_blocks] or NULL (contiguous cache)
   const int32_t* cache_seqlens;    // [B] or NULL
+  int k_add;                       // keys appended after cache_seqlens[b] by this call
   int B, Sq, H, Hkv, G, R;         // R = G * Sq query rows per KV head
   int max_blocks, page_size, num_blocks, seqlen_k_max;
   int unit;                        // tokens per split unit (page or 64)
@@ -53,6 +54,21 @@ struct DecodeParams {
 
 cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           bool bf16, int d, cudaStream_t stream);
+
+// ---------------------------------------------------------------- KV append
+struct AppendParams {
+  void* k_cache;                   // paged pool [num_blocks, page, Hkv, D] or [B, Sk_max, Hkv, D]
+  void* v_cache;
+  const void* k_new;               // [B, S_new, Hkv, D] contiguous
+  const void* v_new;
+  const int32_t* block_table;      // [B, max_blocks] or NULL (contiguous cache)
+  const int32_t* cache_seqlens;    // [B]: keys in the cache before the append
+  int B, S_new, Hkv, D;
+  int max_blocks, page_size, num_blocks, seqlen_k_max;
+  unsigned int* status;
+};
+
+cudaError_t launch_kv_append(const AppendParams& p, cudaStream_t stream);
 
 // ---------------------------------------------------------------- combine
 struct CombineParams {

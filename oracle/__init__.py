@@ -16,6 +16,8 @@ attention(q, k, v, cu_q, cu_k, ...)        dense or varlen (packed rows)
 attention_dense(q, k, v, ...)              [B, S, H, d] convenience form
 attention_paged(q, kpool, vpool, block_table, cache_seqlens, ...)
 combine(out_partial, lse_partial)          LSE-weighted combine of split partials
+append(kcache, vcache, k_new, v_new, cache_seqlens, block_table=None)
+                                           KV-cache append (returns updated copies)
 """
 from __future__ import annotations
 
@@ -185,3 +187,40 @@ def combine(out_partial, lse_partial):
     if rc != 0:
         raise ValueError("oracle_combine: bad arguments")
     return out.reshape(*lead, d), lse.reshape(*lead)
+
+
+def append(kcache, vcache, k_new, v_new, cache_seqlens, block_table=None):
+    """KV-cache append ("flash attention" tag page, section 3.3: with k and v given,
+    flash_attn_with_kvcache writes them into the cache).  Row t of sequence b goes to
+    key position x = cache_seqlens[b] + t, cache_seqlens counting the keys already
+    cached.  Paged cache [num_blocks, page, Hkv, d]: position x of sequence b is row
+    x % page of block block_table[b, x // page]; contiguous cache [B, Sk_max, Hkv, d]:
+    row x of sequence b.  Returns updated copies (inputs untouched) as torch CPU
+    tensors of the caches' dtype; a position outside the cache raises IndexError.
+    Plain element copies, one (b, t) row at a time."""
+    import torch
+    kc = torch.as_tensor(kcache).cpu().clone()
+    vc = torch.as_tensor(vcache).cpu().clone()
+    kn = torch.as_tensor(k_new).cpu()
+    vn = torch.as_tensor(v_new).cpu()
+    cs = [int(x) for x in torch.as_tensor(cache_seqlens).cpu().tolist()]
+    bt = None if block_table is None else torch.as_tensor(block_table).cpu().tolist()
+    B, s_new = kn.shape[0], kn.shape[1]
+    for b in range(B):
+        for t in range(s_new):
+            x = cs[b] + t
+            if bt is not None:
+                page = kc.shape[1]
+                if x < 0 or x // page >= len(bt[b]):
+                    raise IndexError(f"position {x} of sequence {b} is outside the block table")
+                blk = bt[b][x // page]
+                if not 0 <= blk < kc.shape[0]:
+                    raise IndexError(f"block {blk} outside the pool")
+                kc[blk, x % page] = kn[b, t]
+                vc[blk, x % page] = vn[b, t]
+            else:
+                if not 0 <= x < kc.shape[1]:
+                    raise IndexError(f"position {x} of sequence {b} is outside the cache")
+                kc[b, x] = kn[b, t]
+                vc[b, x] = vn[b, t]
+    return kc, vc

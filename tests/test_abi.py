@@ -133,3 +133,40 @@ def test_combine_validation(lib):
 def test_timeout_setter(lib):
     assert lib.fa_set_wait_timeout_ms(0) == FA_ERR_INVALID_ARG
     assert lib.fa_set_wait_timeout_ms(1000) == FA_OK
+
+
+def app(lib, **kw):
+    a = dict(kc=P, vc=P, kn=P, vn=P, dtype=1, B=2, S=1, Hkv=8, d=128, bt=P, maxb=4, page=256,
+             nblk=8, skmax=0, cs=P, stream=None)
+    a.update(kw)
+    return lib.fa_kvcache_append(a["kc"], a["vc"], a["kn"], a["vn"], a["dtype"], a["B"], a["S"],
+                                 a["Hkv"], a["d"], a["bt"], a["maxb"], a["page"], a["nblk"],
+                                 a["skmax"], a["cs"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cs=None), FA_ERR_INVALID_ARG),            # the pre-append lengths are required
+    (dict(dtype=2), FA_ERR_UNSUPPORTED),
+    (dict(d=12), FA_ERR_UNSUPPORTED),
+    (dict(kn=None), FA_ERR_INVALID_ARG),
+    (dict(vc=MIS), FA_ERR_INVALID_ARG),
+    (dict(Hkv=0), FA_ERR_INVALID_ARG),
+    (dict(S=-1), FA_ERR_INVALID_ARG),
+    (dict(page=0), FA_ERR_INVALID_ARG),
+    (dict(bt=None, skmax=-1), FA_ERR_INVALID_ARG),
+])
+def test_append_validation(lib, kw, code):
+    assert app(lib, **kw) == code
+    assert lib.fa_last_error()
+
+
+def test_append_empty_is_a_noop(lib):
+    assert app(lib, B=0) == FA_OK
+    assert app(lib, S=0) == FA_OK
+
+
+def test_fwd_kvcache_append_validation(lib):
+    args = [P, P, P, P, P, 1, P, None, 1, 2, 1, 32, 8, 128, P, 4, 256, 8, 0]
+    tail = [float("nan"), 1, -1, -1, 0.0, None, 1, P, 4096, None]
+    assert lib.fa_fwd_kvcache_append(*args, None, *tail) == FA_ERR_INVALID_ARG   # no cache_seqlens
+    assert lib.fa_fwd_kvcache_append(*args, P, *tail[:-3], None, 0, None) == FA_ERR_WORKSPACE

@@ -373,3 +373,77 @@ def test_generators_are_seeded():
     used = set(bt[bt >= 0].tolist())
     assert len(used) == 3 and all(0 <= x < 5 for x in used)
     assert torch.isnan(kp[int(bt[1, 0]), 20:]).all()
+
+
+# ------------------------------------------------------------------ KV-cache append
+def test_append_hand_positions_paged():
+    """Page 2, sequence 0 holds 1 key, blocks [3, 0]: its two new rows land at key
+    positions 1 and 2 = (block 3, row 1) and (block 0, row 0); sequence 1 holds 2
+    keys, blocks [1, 2]: its rows land at positions 2, 3 = (block 2, rows 0 and 1).
+    Nothing else changes."""
+    kp = torch.zeros(4, 2, 1, 2)
+    vp = torch.zeros(4, 2, 1, 2)
+    bt = torch.tensor([[3, 0, -1], [1, 2, -1]], dtype=torch.int32)
+    cs = torch.tensor([1, 2], dtype=torch.int32)
+    kn = torch.arange(1, 9, dtype=torch.float32).reshape(2, 2, 1, 2)
+    vn = -kn
+    ko, vo = oracle.append(kp, vp, kn, vn, cs, bt)
+    want = torch.zeros(4, 2, 1, 2)
+    want[3, 1, 0] = torch.tensor([1., 2.])
+    want[0, 0, 0] = torch.tensor([3., 4.])
+    want[2, 0, 0] = torch.tensor([5., 6.])
+    want[2, 1, 0] = torch.tensor([7., 8.])
+    assert torch.equal(ko, want)
+    assert torch.equal(vo, -want)
+    assert torch.equal(kp, torch.zeros(4, 2, 1, 2))   # inputs untouched
+
+
+def test_append_hand_positions_contiguous():
+    kc = torch.zeros(2, 4, 1, 1)
+    kn = torch.tensor([[[[5.]], [[6.]]], [[[7.]], [[8.]]]])
+    ko, _ = oracle.append(kc, kc, kn, kn, torch.tensor([0, 2]))
+    assert ko[:, :, 0, 0].tolist() == [[5., 6., 0., 0.], [0., 0., 7., 8.]]
+
+
+def test_append_outside_the_cache_raises():
+    kc = torch.zeros(1, 4, 1, 1)
+    kn = torch.ones(1, 2, 1, 1)
+    with pytest.raises(IndexError):
+        oracle.append(kc, kc, kn, kn, torch.tensor([3]))
+    bt = torch.tensor([[0, 1]], dtype=torch.int32)
+    with pytest.raises(IndexError):
+        oracle.append(torch.zeros(2, 2, 1, 1), torch.zeros(2, 2, 1, 1), kn, kn,
+                      torch.tensor([3]), bt)
+
+
+def test_append_then_attend_equals_attention_on_the_concatenation():
+    """Decoding step of section 3.3: attending the appended cache equals dense
+    attention over (cached keys ++ new keys), the new queries at the last positions."""
+    lens = [5, 16, 0]
+    page, Hkv, d, H, s_new = 8, 2, 8, 4, 3
+    kp, vp, bt, cs = synth.paged_cache(lens, page, Hkv, d, dtype=torch.float32, seed=21,
+                                       spare_blocks=2, tail_fill=0.0)
+    # room for the new rows: fresh zero blocks for the pages they open
+    need = [(L + s_new + page - 1) // page for L in lens]
+    bt = torch.cat([bt, torch.full((len(lens), max(need) - bt.shape[1]), -1,
+                                   dtype=torch.int32)], dim=1)
+    nxt = kp.shape[0]
+    for b, L in enumerate(lens):
+        for pg in range((L + page - 1) // page, need[b]):
+            bt[b, pg] = nxt
+            nxt += 1
+    kp = torch.cat([kp, torch.zeros(nxt - kp.shape[0], page, Hkv, d)])
+    vp = torch.cat([vp, torch.zeros(nxt - vp.shape[0], page, Hkv, d)])
+    g = torch.Generator().manual_seed(22)
+    kn = torch.randn(3, s_new, Hkv, d, generator=g)
+    vn = torch.randn(3, s_new, Hkv, d, generator=g)
+    q = torch.randn(3, s_new, H, d, generator=g)
+    ka, va = oracle.append(kp, vp, kn, vn, cs, bt)
+    out, lse = oracle.attention_paged(q, ka, va, bt, cs + s_new, causal=True)
+    for b, L in enumerate(lens):
+        rows = [int(bt[b, j // page]) * page + j % page for j in range(L)]
+        kc = torch.cat([kp.reshape(-1, Hkv, d)[rows], kn[b]])[None]
+        vc = torch.cat([vp.reshape(-1, Hkv, d)[rows], vn[b]])[None]
+        o1, l1 = oracle.attention_dense(q[b:b + 1], kc, vc, causal=True)
+        np.testing.assert_allclose(out[b], o1[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b], l1[0], rtol=0, atol=1e-12)
