@@ -117,7 +117,8 @@ FA_API int fa_kvcache_num_splits(int batch, int seqlen_q, int num_heads, int num
  * fa_kvcache_workspace_size -- bytes of device scratch fa_fwd_kvcache needs:
  * 256 (a work-item counter the call resets) plus, when the resolved split count is
  * above 1, splits * batch * seqlen_q * num_heads * (head_dim + 1) * 4 for the fp32
- * split partials.  Same arguments as fa_kvcache_num_splits.
+ * split partials.  Same arguments as fa_kvcache_num_splits (which returns 1 when
+ * the call runs the tensor-core kernel: more than 16 query rows per KV head).
  */
 FA_API size_t fa_kvcache_workspace_size(int batch, int seqlen_q, int num_heads, int num_heads_k,
                                  int head_dim, int max_seqlen_k, int page_size,
@@ -151,7 +152,13 @@ FA_API size_t fa_kvcache_workspace_size(int batch, int seqlen_q, int num_heads, 
  *   (zeroed by the call with an asynchronous memset on `stream`) and the fp32
  *   split partials between the two kernels of one call, so calls that share a
  *   workspace must be stream-ordered.
- * Limits: num_heads / num_heads_k * seqlen_q <= 16 rows per KV head.
+ * Up to 16 query rows per KV head ((num_heads / num_heads_k) * seqlen_q) the call
+ *   runs the split-KV decode kernel above.  With more (chunked prefill against the
+ *   cache: a chunk of new query rows attends everything cached, causal aligned
+ *   bottom-right) it runs the tcgen05 prefill kernel of fa_fwd with K/V read from
+ *   the cache, one CTA per 256 query rows; num_splits is then ignored.  Keys past
+ *   a sequence's length (page tails, unused blocks) are never loaded or are
+ *   cleared before use, so their contents cannot reach the output either way.
  */
 FA_API int fa_fwd_kvcache(const void *q, const void *k_cache, const void *v_cache, void *out, float *lse,
                    int dtype, int batch, int seqlen_q, int num_heads, int num_heads_k,

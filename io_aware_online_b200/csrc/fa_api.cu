@@ -305,8 +305,18 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
   return FA_OK;
 }
 
+// Query rows per KV head above which fa_fwd_kvcache runs the tensor-core prefill
+// kernel over the cache instead of the split-KV decode kernel.
+static constexpr int kDecodeMaxRows = 16;
+
+static bool kvcache_uses_prefill(int seqlen_q, int num_heads, int num_heads_k) {
+  return num_heads_k > 0 &&
+         static_cast<long>(num_heads / num_heads_k) * seqlen_q > kDecodeMaxRows;
+}
+
 int fa_kvcache_num_splits(int batch, int seqlen_q, int num_heads, int num_heads_k, int head_dim,
                           int max_seqlen_k, int page_size, int num_splits) {
+  if (kvcache_uses_prefill(seqlen_q, num_heads, num_heads_k)) return 1;  // no split partials
   const int unit = page_size > 0 ? page_size : 64;
   return resolve_splits(batch, seqlen_q, num_heads, num_heads_k, head_dim, max_seqlen_k, unit,
                         num_splits);
@@ -346,9 +356,7 @@ static int kvcache_impl(const void* q, const void* k_cache, const void* v_cache,
   if (batch < 0 || seqlen_q < 0 || num_splits < 0)
     return fail(FA_ERR_INVALID_ARG, "fa_fwd_kvcache: negative size");
   const int H = num_heads, Hkv = num_heads_k, d = head_dim, G = H / Hkv;
-  if (static_cast<long>(G) * seqlen_q > 16)
-    return fail(FA_ERR_UNSUPPORTED, "fa_fwd_kvcache: (num_heads/num_heads_k)*seqlen_q = %ld > 16 rows per KV head",
-                static_cast<long>(G) * seqlen_q);
+  const bool use_prefill = kvcache_uses_prefill(seqlen_q, H, Hkv);
   const bool paged = block_table != nullptr;
   int max_k, unit;
   if (paged) {
@@ -378,7 +386,6 @@ static int kvcache_impl(const void* q, const void* k_cache, const void* v_cache,
     const cudaError_t e0 = fa::launch_kv_append(*app, static_cast<cudaStream_t>(stream));
     return e0 == cudaSuccess ? FA_OK : cuda_fail(e0, "fa_fwd_kvcache_append append launch");
   }
-  const int splits = resolve_splits(batch, seqlen_q, H, Hkv, d, max_k, unit, num_splits);
   const size_t need = fa_kvcache_workspace_size(batch, seqlen_q, H, Hkv, d, max_k,
                                                 paged ? page_size : 0, num_splits);
   if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
@@ -388,6 +395,68 @@ static int kvcache_impl(const void* q, const void* k_cache, const void* v_cache,
   unsigned int* status = nullptr;
   int sms = 0;
   if ((rc = device_state(nullptr, &status, &sms)) != FA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (app != nullptr) app->status = status;
+
+  if (use_prefill) {
+    // many query rows per KV head (chunked prefill against the cache): the tcgen05
+    // prefill kernel, K/V read from the cache in 64-row boxes
+    if (seqlen_q > 65535 * 128)
+      return fail(FA_ERR_UNSUPPORTED, "fa_fwd_kvcache: seqlen_q %d too large", seqlen_q);
+    CUtensorMap tq, tk, tv;
+    {
+      const uint32_t box[4] = {64, 128, 1, 1};
+      const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(seqlen_q),
+                                static_cast<uint64_t>(H), static_cast<uint64_t>(batch)};
+      const uint64_t st[3] = {static_cast<uint64_t>(H) * d * 2, static_cast<uint64_t>(d) * 2,
+                              static_cast<uint64_t>(seqlen_q) * H * d * 2};
+      if ((rc = encode_4d(&tq, q, dims, st, box, "q")) != FA_OK) return rc;
+    }
+    {
+      const uint32_t box[4] = {64, 64, 1, 1};
+      const uint64_t rows = paged ? page_size : std::max(seqlen_k_max, 1);
+      const uint64_t dims[4] = {static_cast<uint64_t>(d), rows, static_cast<uint64_t>(Hkv),
+                                static_cast<uint64_t>(paged ? num_blocks : batch)};
+      const uint64_t st[3] = {static_cast<uint64_t>(Hkv) * d * 2, static_cast<uint64_t>(d) * 2,
+                              rows * Hkv * d * 2};
+      if ((rc = encode_4d(&tk, k_cache, dims, st, box, "k_cache")) != FA_OK) return rc;
+      if ((rc = encode_4d(&tv, v_cache, dims, st, box, "v_cache")) != FA_OK) return rc;
+    }
+    fa::FwdParams f{};
+    f.out = out;
+    f.lse = lse;
+    f.o_sb = static_cast<int64_t>(seqlen_q) * H * d;
+    f.o_ss = static_cast<int64_t>(H) * d;
+    f.o_sh = d;
+    f.Sq = seqlen_q;
+    f.Sk = paged ? 0 : seqlen_k_max;
+    f.H = H;
+    f.G = G;
+    f.total_q = seqlen_q;
+    fill_score_params(scale, softcap, &f.scale_log2, &f.softcap_log2, &f.tanh_k);
+    f.alibi = alibi_slopes;
+    f.causal = causal ? 1 : 0;
+    f.wl = window_left;
+    f.wr = window_right;
+    f.tile_major = (!causal && window_left < 0 && window_right < 0) ? 1 : 0;
+    f.status = status;
+    f.timeout_ns = timeout_ns();
+    f.kv_mode = 1;
+    f.block_table = block_table;
+    f.cache_seqlens = cache_seqlens;
+    f.k_add = app ? app->S_new : 0;
+    f.page_size = page_size;
+    f.max_blocks = max_blocks_per_seq;
+    f.num_blocks = num_blocks;
+    cudaError_t e = cudaSuccess;
+    if (app != nullptr && (e = fa::launch_kv_append(*app, s)) != cudaSuccess)
+      return cuda_fail(e, "fa_fwd_kvcache_append append launch");
+    e = (dtype == FA_BF16) ? fa::launch_fwd_bf16(tq, tk, tv, f, d, batch, seqlen_q, s)
+                           : fa::launch_fwd_f16(tq, tk, tv, f, d, batch, seqlen_q, s);
+    if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache prefill launch");
+    return FA_OK;
+  }
+  const int splits = resolve_splits(batch, seqlen_q, H, Hkv, d, max_k, unit, num_splits);
 
   CUtensorMap tk, tv;
   const uint32_t box[4] = {64, 1, 64, 1};
@@ -441,10 +510,8 @@ static int kvcache_impl(const void* q, const void* k_cache, const void* v_cache,
   p.status = status;
   p.timeout_ns = timeout_ns();
   p.sm_count = sms;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (app != nullptr) {
-    app->status = status;
     e = fa::launch_kv_append(*app, s);
     if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache_append append launch");
   }

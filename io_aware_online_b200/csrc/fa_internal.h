@@ -24,6 +24,13 @@ struct FwdParams {
   const float* alibi;              // [H] or NULL
   int causal, wl, wr;              // mask flags; -1 = unbounded window side
   int tile_major;                  // grid x = query tiles (no mask: equal work per tile)
+  // KV-cache mode (fa_fwd_kvcache with many query rows): K/V come from a paged pool
+  // [num_blocks, page, Hkv, D] through block_table, or from a contiguous cache
+  // [B, Sk, Hkv, D], in 64-row boxes; sequence b attends cache_seqlens[b] + k_add keys
+  int kv_mode;
+  const int32_t* block_table;      // [B, max_blocks] or NULL (contiguous cache)
+  const int32_t* cache_seqlens;    // [B] or NULL (= Sk)
+  int k_add, page_size, max_blocks, num_blocks;
   unsigned int* status;            // device status word
   uint64_t timeout_ns;             // bounded-wait limit
 };

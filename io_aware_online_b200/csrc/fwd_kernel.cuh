@@ -153,6 +153,14 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
     Sq_b = p.cu_q[b + 1] - q0;
     k0 = p.cu_k[b];
     Sk_b = p.cu_k[b + 1] - k0;
+  } else if (p.kv_mode) {
+    Sk_b = ((p.cache_seqlens != nullptr) ? p.cache_seqlens[b] : p.Sk) + p.k_add;
+    // a length the cache cannot hold would read past the block table: clamp, report
+    const int cap = (p.block_table != nullptr) ? p.max_blocks * p.page_size : p.Sk;
+    if (Sk_b < 0 || Sk_b > cap) {
+      if (threadIdx.x == 0) atomicOr(p.status, kDevBadLength);
+      Sk_b = min(max(Sk_b, 0), cap);
+    }
   }
   const int n_units_b = (Sq_b + T * kBM - 1) / (T * kBM);
   if (zi >= n_units_b) return;  // uniform: whole CTA leaves
@@ -242,18 +250,57 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
         const int s = it % ST;
         const uint32_t ph = (it / ST) & 1;
         const int j = j_lo + it;
-        if (!wait_bounded(k_empty + s, ph ^ 1, w)) break;
-        mbar_arrive_expect_tx(k_full + s, Cfg::kTileBytes);
-        for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_4d(sK + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmK, k_full + s, c * 64,
-                      krow + j * kBN, hk, b_coord);
-        last_k[s] = ph;
-        if (!wait_bounded(v_empty + s, ph ^ 1, w)) break;
-        mbar_arrive_expect_tx(v_full + s, Cfg::kTileBytes);
-        for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_4d(sV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmV, v_full + s, c * 64,
-                      krow + j * kBN, hk, b_coord);
-        last_v[s] = ph;
+        if (!p.kv_mode) {
+          if (!wait_bounded(k_empty + s, ph ^ 1, w)) break;
+          mbar_arrive_expect_tx(k_full + s, Cfg::kTileBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_4d(sK + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmK, k_full + s,
+                        c * 64, krow + j * kBN, hk, b_coord);
+          last_k[s] = ph;
+          if (!wait_bounded(v_empty + s, ph ^ 1, w)) break;
+          mbar_arrive_expect_tx(v_full + s, Cfg::kTileBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_4d(sV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmV, v_full + s,
+                        c * 64, krow + j * kBN, hk, b_coord);
+          last_v[s] = ph;
+        } else {
+          // KV cache: the block's two 64-key halves, each inside one page (page_size
+          // is a multiple of 64); halves at or past the sequence's end are not
+          // loaded (their rows are masked, and V's are zeroed before P.V)
+          int row[2], blk[2], nh = 0;
+          for (int hh = 0; hh < 2; ++hh) {
+            const int pos = j * kBN + hh * 64;
+            if (pos >= Sk_b) break;
+            if (p.block_table != nullptr) {
+              int bk = p.block_table[static_cast<int64_t>(b) * p.max_blocks + pos / p.page_size];
+              if (bk < 0 || bk >= p.num_blocks) {
+                atomicOr(p.status, kDevBadBlock);
+                bk = 0;  // read a valid page; the status word reports the fault
+              }
+              row[hh] = pos % p.page_size;
+              blk[hh] = bk;
+            } else {
+              row[hh] = pos;
+              blk[hh] = b;
+            }
+            ++nh;
+          }
+          constexpr uint32_t kHalfBytes = Cfg::kChunks * 64 * 128;
+          if (!wait_bounded(k_empty + s, ph ^ 1, w)) break;
+          mbar_arrive_expect_tx(k_full + s, nh * kHalfBytes);
+          for (int hh = 0; hh < nh; ++hh)
+            for (int c = 0; c < Cfg::kChunks; ++c)
+              tma_load_4d(sK + s * Cfg::kTileBytes + c * Cfg::kChunkBytes + hh * 64 * 128, &tmK,
+                          k_full + s, c * 64, row[hh], hk, blk[hh]);
+          last_k[s] = ph;
+          if (!wait_bounded(v_empty + s, ph ^ 1, w)) break;
+          mbar_arrive_expect_tx(v_full + s, nh * kHalfBytes);
+          for (int hh = 0; hh < nh; ++hh)
+            for (int c = 0; c < Cfg::kChunks; ++c)
+              tma_load_4d(sV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes + hh * 64 * 128, &tmV,
+                          v_full + s, c * 64, row[hh], hk, blk[hh]);
+          last_v[s] = ph;
+        }
       }
       if (*abort_flag) {  // let this CTA's own copies land before the smem goes away
         wait_drain(q_full, 0, p.timeout_ns);
@@ -567,6 +614,27 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
           tmem_st32(tO + c * 32, o);
         }
+      }
+      // KV cache, last block of the sequence: V rows past its end hold whatever
+      // the page tail (or an unloaded half) holds; P is 0 there, but 0 * NaN is
+      // NaN in P.V, so this warp zeroes its 32 rows of them before releasing P
+      // (both tiles' warps write the same zeros)
+      if (p.kv_mode && kb + kBN > Sk_b) {
+        const int s = it % ST;
+        ok = wait_bounded(v_full + s, (it / ST) & 1, w);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        if (kb + r >= Sk_b) {
+          uint8_t* vrow = sV + s * Cfg::kTileBytes + r * 128;
+#pragma unroll
+          for (int c = 0; c < Cfg::kChunks; ++c)
+#pragma unroll
+            for (int v16 = 0; v16 < 8; ++v16)
+              reinterpret_cast<uint4*>(vrow + c * Cfg::kChunkBytes)[v16] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
       }
       tmem_st_wait();
       tc_fence_before();

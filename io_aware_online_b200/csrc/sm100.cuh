@@ -90,6 +90,12 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, con
   return wait_slow(bar, parity, w);
 }
 
+// Orders this thread's generic-proxy shared-memory writes before later async-proxy
+// (TMA, tcgen05.mma) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -104,7 +104,6 @@ def kvc(lib, **kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(page=100), FA_ERR_INVALID_ARG),
     (dict(cs=None), FA_ERR_INVALID_ARG),            # paged cache needs cache_seqlens
-    (dict(Sq=5), FA_ERR_UNSUPPORTED),               # 4 * 5 = 20 rows per KV head > 16
     (dict(nblk=0), FA_ERR_INVALID_ARG),
     (dict(d=80), FA_ERR_UNSUPPORTED),
     (dict(splits=4, ws=None, wsb=0), FA_ERR_WORKSPACE),
@@ -121,6 +120,9 @@ def test_splits_and_workspace_size(lib):
     assert lib.fa_kvcache_num_splits(64, 1, 32, 8, 128, 512, 256, 16) == 2
     assert lib.fa_kvcache_workspace_size(64, 1, 32, 8, 128, 32768, 256, 1) == 256
     assert lib.fa_kvcache_workspace_size(64, 1, 32, 8, 128, 32768, 256, 4) == 256 + 4 * 64 * 32 * 129 * 4
+    # more than 16 query rows per KV head run the tensor-core kernel: no split partials
+    assert lib.fa_kvcache_num_splits(4, 128, 32, 8, 128, 32768, 256, 16) == 1
+    assert lib.fa_kvcache_workspace_size(4, 128, 32, 8, 128, 32768, 256, 16) == 256
 
 
 def test_combine_validation(lib):
