@@ -321,6 +321,96 @@ def run_ours(args, rank, world, local):
     return res
 
 
+# Workloads of the cache-update rows (not part of the default step): a 2048-token
+# chunk appended after 6144 cached tokens and attended causally (chunked prefill),
+# and a whole 8192-token prompt written into an empty paged cache (append).
+CHUNKED = dict(B=4, cached=6144, chunk=2048, H=32, Hkv=8, d=128, dtype="bf16", page=256)
+APPEND = dict(B=4, S_new=8192, Hkv=8, d=128, dtype="bf16", page=256)
+
+
+def run_cache_rows(args, rank, world, local):
+    """--only chunked | append: time one cache-update row on its own workload."""
+    import io_aware_online_b200 as fa
+    from io_aware_online_b200 import build as fa_build
+    fa_build.build()
+    fa.load()
+    dev = torch.device("cuda", local)
+    hbm_peak, tflops_peak, peak_src = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    c = CHUNKED if args.only == "chunked" else APPEND
+    dt = synth.DTYPES[c["dtype"]]
+    B, Hkv, d, page = c["B"], c["Hkv"], c["d"], c["page"]
+    s_new = c["chunk"] if args.only == "chunked" else c["S_new"]
+    cached = c.get("cached", 0)
+    total = cached + s_new
+    nblk = (total + page - 1) // page
+    gen = torch.Generator(device=dev).manual_seed(3000 + rank)
+    kp = torch.randn(B * nblk, page, Hkv, d, generator=gen, device=dev).to(dt)
+    vp = torch.randn(B * nblk, page, Hkv, d, generator=gen, device=dev).to(dt)
+    perm = torch.randperm(B * nblk, generator=torch.Generator().manual_seed(3001 + rank))
+    bt = perm.to(torch.int32).reshape(B, nblk).to(dev)
+    cs = torch.full((B,), cached, dtype=torch.int32, device=dev)
+    kn = torch.randn(B, s_new, Hkv, d, generator=gen, device=dev).to(dt)
+    vn = torch.randn(B, s_new, Hkv, d, generator=gen, device=dev).to(dt)
+    if args.only == "chunked":
+        H = c["H"]
+        q = torch.randn(B, s_new, H, d, generator=gen, device=dev).to(dt)
+        out = torch.empty_like(q)
+        lse = torch.empty((B, H, s_new), dtype=torch.float32, device=dev)
+        ws = torch.empty(256, dtype=torch.uint8, device=dev)
+        pairs = sum(cached + i + 1 for i in range(s_new))
+        work = 4.0 * d * H * B * pairs                      # algorithmic FLOPs
+
+        def call():
+            fa.fa_fwd_kvcache(q, kp, vp, kn, vn, cache_seqlens=cs, block_table=bt, causal=True,
+                              out=out, lse=lse, workspace=ws, stream=stream)
+    else:
+        work = 2.0 * B * s_new * Hkv * d * 2 * 2            # bytes: K and V, read and written
+
+        def call():
+            fa.fa_kvcache_append(kp, vp, kn, vn, cs, block_table=bt, stream=stream)
+    for _ in range(args.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with Clocks(dev.index if dev.index is not None else 0) as clk:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world)
+    if args.only == "chunked":
+        achieved = work / (ms * 1e-3) / 1e12
+        metric, unit, peak, punit, bound = ("chunked prefill TFLOPS (append + attend, paged KV "
+                                            "cache)", "TFLOPS", tflops_peak, "TFLOP/s", "tensor")
+        kernel = "kv_append_kernel + fwd_kernel<128, bf16, causal> in KV-cache mode"
+    else:
+        achieved = work / (ms * 1e-3) / 1e9
+        metric, unit, peak, punit, bound = ("KV-cache append GB/s (paged)", "GB/s", hbm_peak,
+                                            "GB/s", "hbm")
+        kernel = "kv_append_kernel"
+    value = achieved * world
+    return {"metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": c["dtype"], "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": args.only, **c, "l2": "flushed between steps (256 MiB write, "
+                       "untimed)", "parallelism": f"dp{world} (independent replicas)"},
+            "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak,
+                         "unit": punit, "frac": round(achieved / peak, 4), "traffic": None,
+                         "kernel": kernel, "peak_source": peak_src},
+            "gpu_launches": K * (2 if args.only == "chunked" else 1),
+            "clocks": clk.summary()}
+
+
 def e2e_prefill(fa, q, k, v, dev, stream, flops, world, steps=5):
     """Prefill TFLOPS through the public call with pinned host buffers: the H2D copy
     of q, k, v, the kernel and the D2H copy of O are all inside the timed region."""
@@ -410,8 +500,10 @@ def main():
     ap.add_argument("--num-splits", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
-                    help="time one part of the step (profiling / sweeps)")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "chunked", "append"],
+                    default="all",
+                    help="time one part of the step (profiling / sweeps), or one of the "
+                         "cache-update rows on its own workload (chunked, append)")
     ap.add_argument("--prefill-seq", type=int, default=PREFILL["S"])
     ap.add_argument("--prefill-d", type=int, default=PREFILL["d"])
     ap.add_argument("--prefill-dtype", choices=["fp16", "bf16"], default=PREFILL["dtype"])
@@ -426,6 +518,11 @@ def main():
         if args.impl == "reference":
             if rank == 0:
                 print(json.dumps(run_reference(args, rank, world)), flush=True)
+            return
+        if args.only in ("chunked", "append"):
+            res = run_cache_rows(args, rank, world, local)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
             return
         res = run_ours(args, rank, world, local)
         if rank == 0:
