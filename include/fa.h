@@ -217,6 +217,17 @@ FA_API int fa_fwd_kvcache_append(const void *q, void *k_cache, void *v_cache, co
                                  void *stream);
 
 /*
+ * fa_selftest_wait_timeout -- a diagnostic of the bounded waits (the pages have no
+ * counterpart): launches one CTA that waits, through the library's bounded wait, on
+ * a barrier phase nothing ever completes.  After timeout_ms (1..10000) of GPU time
+ * the wait gives up and raises FA_DEV_WAIT_TIMEOUT in the device status word, as a
+ * stalled pipeline wait of any kernel here would; read it with fa_device_status
+ * after synchronising `stream`.  The context stays usable.  Returns FA_OK once
+ * launched, FA_ERR_INVALID_ARG for a limit out of range.
+ */
+FA_API int fa_selftest_wait_timeout(int timeout_ms, void *stream);
+
+/*
  * fa_fwd_kvcache_static -- fa_fwd_kvcache without a workspace argument, for callers
  * that cannot allocate device memory where they run attention (a host framework
  * that owns every device allocation through its own pool, or a serving loop that

@@ -87,6 +87,8 @@ def load():
     lib.fa_device_status.restype = i32
     lib.fa_set_wait_timeout_ms.argtypes = [i32]
     lib.fa_set_wait_timeout_ms.restype = i32
+    lib.fa_selftest_wait_timeout.argtypes = [i32, vp]
+    lib.fa_selftest_wait_timeout.restype = i32
     lib.fa_version.argtypes = []
     lib.fa_version.restype = i32
     _lib = lib
@@ -324,3 +326,9 @@ def fa_combine(out_partial, lse_partial, *, out_dtype=torch.float32, out=None, l
                           _DT[out.dtype], B, S, H, d, splits, _i64(out_partial.stride()),
                           _i64(lse_partial.stride()), _stream(stream)))
     return out, lse
+
+
+def fa_selftest_wait_timeout(timeout_ms=20, stream=None):
+    """Launch the bounded-wait self-test (include/fa.h): after timeout_ms the waiting
+    CTA raises FA_DEV_WAIT_TIMEOUT in the device status word and exits."""
+    _check(load().fa_selftest_wait_timeout(int(timeout_ms), _stream(stream)))

@@ -547,6 +547,18 @@ static int kvcache_impl(const void* q, const void* k_cache, const void* v_cache,
   return FA_OK;
 }
 
+int fa_selftest_wait_timeout(int timeout_ms, void* stream) {
+  g_err.clear();
+  if (timeout_ms <= 0 || timeout_ms > 10000)
+    return fail(FA_ERR_INVALID_ARG, "fa_selftest_wait_timeout: timeout_ms must be in 1..10000");
+  unsigned int* status = nullptr;
+  int rc = device_state(nullptr, &status, nullptr);
+  if (rc != FA_OK) return rc;
+  const cudaError_t e = fa::launch_wait_timeout_selftest(
+      status, static_cast<uint64_t>(timeout_ms) * 1000000ull, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e, "fa_selftest_wait_timeout launch");
+}
+
 int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void* out, float* lse,
                    int dtype, int batch, int seqlen_q, int num_heads, int num_heads_k,
                    int head_dim, const int32_t* block_table, int max_blocks_per_seq,

@@ -91,6 +91,9 @@ struct CombineParams {
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
+cudaError_t launch_wait_timeout_selftest(unsigned int* status, uint64_t timeout_ns,
+                                         cudaStream_t stream);
+
 // Sets the calling thread's fa_last_error() message; returns `code`.
 int set_error(int code, const char* msg);
 

@@ -172,3 +172,8 @@ def test_fwd_kvcache_append_validation(lib):
     tail = [float("nan"), 1, -1, -1, 0.0, None, 1, P, 4096, None]
     assert lib.fa_fwd_kvcache_append(*args, None, *tail) == FA_ERR_INVALID_ARG   # no cache_seqlens
     assert lib.fa_fwd_kvcache_append(*args, P, *tail[:-3], None, 0, None) == FA_ERR_WORKSPACE
+
+
+def test_selftest_limit_validation(lib):
+    assert lib.fa_selftest_wait_timeout(0, None) == FA_ERR_INVALID_ARG
+    assert lib.fa_selftest_wait_timeout(20000, None) == FA_ERR_INVALID_ARG
