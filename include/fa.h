@@ -18,7 +18,7 @@
  *   nothing was launched.
  * - Dtypes: FA_FP16 or FA_BF16 for Q, K, V and O (one dtype per call); LSE,
  *   ALiBi slopes and split partials are fp32.  fp32 inputs are not supported
- *   (the pages: fp16/bf16 only).
+ *   (the pages: fp16/bf16 only).  fa_fwd_fp8 takes E4M3 Q, K, V and writes bf16.
  * - Head dim: 64 or 128.
  * - softmax_scale: a NaN means the default 1/sqrt(head_dim) (section 3.1);
  *   otherwise it must be finite and >= 0.
@@ -102,6 +102,36 @@ FA_API int fa_fwd(const void *q, const void *k, const void *v, void *out, float 
            const int64_t *o_strides, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
            int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal, int window_left,
            int window_right, float softcap, const float *alibi_slopes, void *stream);
+
+/*
+ * fa_fwd_fp8 -- fa_fwd with 8-bit inputs (the "FlashAttention common interfaces"
+ * page's workflow three: q, k and v cast to float8 E4M3 and passed to the same
+ * call; FlashAttention-3's FP8 path on the tag page).
+ *
+ *   q, k, v: E4M3 bytes, layouts and strides (in elements, multiples of 16) as for
+ *   fa_fwd; head_dim must be 128.  out: bf16, layout as for fa_fwd (strides in
+ *   elements, multiples of 8).  lse: fp32 as for fa_fwd, or NULL.
+ *   q_descale, k_descale, v_descale: finite, > 0 (1 for a plain cast): the real
+ *   inputs are q * q_descale etc.; the scores use softmax_scale * q_descale *
+ *   k_descale and O is multiplied by v_descale.
+ * Both products run on the tensor cores with 8-bit operands (tcgen05.mma
+ * kind::f8f6f4), so P is rounded to E4M3 before P.V: each probability carries a
+ * relative error of at most 2^-4, and O differs from exact attention on the
+ * dequantised inputs by at most 2^-4 * sum_j w_ij |v_j| per element (w the exact
+ * attention weights) plus n_k * 2^-18 * max_j |v_j| (probabilities below 2^-14 of
+ * the row's largest fall in E4M3's subnormal range), plus the bf16 rounding of O.
+ * The LSE comes from the exact fp32 sum.  Other arguments, masks and errors as for
+ * fa_fwd.
+ */
+FA_API int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out, float *lse,
+                      float q_descale, float k_descale, float v_descale, int batch,
+                      int seqlen_q, int seqlen_k, int num_heads, int num_heads_k, int head_dim,
+                      const int64_t *q_strides, const int64_t *k_strides,
+                      const int64_t *v_strides, const int64_t *o_strides,
+                      const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                      int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal,
+                      int window_left, int window_right, float softcap,
+                      const float *alibi_slopes, void *stream);
 
 /*
  * fa_kvcache_num_splits -- the split count fa_fwd_kvcache uses for these sizes.

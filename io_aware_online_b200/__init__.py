@@ -58,6 +58,10 @@ def load():
     lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i64p, i64p,
                            i64p, i64p, vp, vp, i32, i32, f32, i32, i32, i32, f32, vp, vp]
     lib.fa_fwd.restype = i32
+    lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, f32, f32, f32, i32, i32, i32, i32, i32, i32,
+                               i64p, i64p, i64p, i64p, vp, vp, i32, i32, f32, i32, i32, i32, f32,
+                               vp, vp]
+    lib.fa_fwd_fp8.restype = i32
     lib.fa_kvcache_num_splits.argtypes = [i32] * 8
     lib.fa_kvcache_num_splits.restype = i32
     lib.fa_kvcache_workspace_size.argtypes = [i32] * 8
@@ -144,7 +148,8 @@ def fa_device_status(clear: bool = True) -> int:
 
 def fa_fwd(q, k, v, *, out=None, lse=None, cu_seqlens_q=None, cu_seqlens_k=None,
            max_seqlen_q=None, max_seqlen_k=None, softmax_scale=None, causal=False,
-           window_size=(-1, -1), softcap=0.0, alibi_slopes=None, return_lse=True, stream=None):
+           window_size=(-1, -1), softcap=0.0, alibi_slopes=None, return_lse=True, stream=None,
+           _fp8=None):
     """Exact attention forward (sections 3.1 / 3.2 of the interface page).
 
     Dense: q [B, Sq, H, d], k/v [B, Sk, Hkv, d] -> out like q, lse [B, H, Sq].
@@ -152,7 +157,8 @@ def fa_fwd(q, k, v, *, out=None, lse=None, cu_seqlens_q=None, cu_seqlens_k=None,
     max_seqlen_q/k -> out like q, lse [H, total_q].
     """
     lib = load()
-    dt = _dtype(q)
+    fp8 = _fp8
+    dt = _DT[torch.bfloat16] if fp8 is not None else _dtype(q)
     varlen = cu_seqlens_q is not None or cu_seqlens_k is not None
     if varlen:
         total_q, H, d = q.shape
@@ -181,12 +187,29 @@ def fa_fwd(q, k, v, *, out=None, lse=None, cu_seqlens_q=None, cu_seqlens_k=None,
     if lse is None and return_lse:
         shape = (H, sq) if varlen else (B, H, sq)
         lse = torch.empty(shape, dtype=torch.float32, device=q.device)
-    _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), dt, B, sq, sk, H, Hkv, d,
-                      _i64(qs), _i64(ks), _i64(vs), _i64(os_), _ptr(cu_seqlens_q),
-                      _ptr(cu_seqlens_k), int(max_seqlen_q), int(max_seqlen_k),
-                      _scale(softmax_scale), int(bool(causal)), int(window_size[0]),
-                      int(window_size[1]), float(softcap), _ptr(alibi_slopes), _stream(stream)))
+    args = (_i64(qs), _i64(ks), _i64(vs), _i64(os_), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+            int(max_seqlen_q), int(max_seqlen_k), _scale(softmax_scale), int(bool(causal)),
+            int(window_size[0]), int(window_size[1]), float(softcap), _ptr(alibi_slopes),
+            _stream(stream))
+    if fp8 is None:
+        _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), dt, B, sq, sk, H, Hkv,
+                          d, *args))
+    else:
+        _check(lib.fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), *fp8, B, sq, sk,
+                              H, Hkv, d, *args))
     return out, lse
+
+
+def fa_fwd_fp8(q, k, v, *, q_descale=1.0, k_descale=1.0, v_descale=1.0, **kw):
+    """fa_fwd on float8_e4m3fn q, k, v (head_dim 128) with per-tensor descale
+    factors (the real inputs are q * q_descale etc.); out is bf16.  Other keywords
+    as for fa_fwd."""
+    for t in (q, k, v):
+        if t.dtype != torch.float8_e4m3fn:
+            raise TypeError("fa_fwd_fp8 takes float8_e4m3fn q, k, v")
+    if kw.get("out") is None:
+        kw["out"] = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    return fa_fwd(q, k, v, _fp8=(float(q_descale), float(k_descale), float(v_descale)), **kw)
 
 
 def fa_kvcache_num_splits(batch, seqlen_q, num_heads, num_heads_k, head_dim, max_seqlen_k,

@@ -24,6 +24,8 @@ cudaError_t launch_fwd_f16(const CUtensorMap&, const CUtensorMap&, const CUtenso
                            const FwdParams&, int, int, int, cudaStream_t);
 cudaError_t launch_fwd_bf16(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                             const FwdParams&, int, int, int, cudaStream_t);
+cudaError_t launch_fwd_fp8(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                           const FwdParams&, int, int, int, cudaStream_t);
 }  // namespace fa
 
 // Device status word: kernels OR FA_DEV_* bits into it; fa_device_status reads it.
@@ -106,7 +108,8 @@ int get_encoder() {
 
 // 4-D tiled map over 16-bit elements, 128-byte swizzle (box inner extent 64).
 int encode_4d(CUtensorMap* map, const void* ptr, const uint64_t dims[4],
-              const uint64_t strides_bytes[3], const uint32_t box[4], const char* what) {
+              const uint64_t strides_bytes[3], const uint32_t box[4], const char* what,
+              bool bytes = false) {
   for (int i = 0; i < 3; ++i)
     if (strides_bytes[i] % 16 != 0 || strides_bytes[i] >= (1ull << 40) || strides_bytes[i] == 0)
       return fail(FA_ERR_INVALID_ARG, "%s: stride %d (%llu bytes) must be a positive multiple of 16",
@@ -115,7 +118,8 @@ int encode_4d(CUtensorMap* map, const void* ptr, const uint64_t dims[4],
   cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
   cuuint64_t gs[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
   cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(ptr), gd, gs, bx,
+  CUresult r = g_encode(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                        4, const_cast<void*>(ptr), gd, gs, bx,
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FA_ERR_INVALID_ARG, "%s: tensor map encoding failed (%d)", what, (int)r);
@@ -211,15 +215,24 @@ int fa_device_status(int clear, unsigned int* flags) {
   return FA_OK;
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int dtype,
-           int batch, int seqlen_q, int seqlen_k, int num_heads, int num_heads_k, int head_dim,
-           const int64_t* q_strides, const int64_t* k_strides, const int64_t* v_strides,
-           const int64_t* o_strides, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
-           int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal, int window_left,
-           int window_right, float softcap, const float* alibi_slopes, void* stream) {
-  g_err.clear();
-  int rc = check_common(dtype, head_dim, num_heads, num_heads_k, window_left, window_right, softcap);
+// fa_fwd's body; fp8: E4M3 q, k, v (head_dim 128), bf16 output, per-tensor descales.
+static int fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int dtype,
+                    int batch, int seqlen_q, int seqlen_k, int num_heads, int num_heads_k,
+                    int head_dim, const int64_t* q_strides, const int64_t* k_strides,
+                    const int64_t* v_strides, const int64_t* o_strides,
+                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int max_seqlen_q,
+                    int max_seqlen_k, float softmax_scale, int causal, int window_left,
+                    int window_right, float softcap, const float* alibi_slopes, void* stream,
+                    bool fp8, float q_descale, float k_descale, float v_descale) {
+  int rc = check_common(fp8 ? FA_BF16 : dtype, head_dim, num_heads, num_heads_k, window_left,
+                        window_right, softcap);
   if (rc != FA_OK) return rc;
+  if (fp8 && head_dim != 128)
+    return fail(FA_ERR_UNSUPPORTED, "fa_fwd_fp8: head_dim %d (8-bit inputs need 128)", head_dim);
+  if (fp8 && (!(q_descale > 0.f) || !(k_descale > 0.f) || !(v_descale > 0.f) ||
+              std::isinf(q_descale) || std::isinf(k_descale) || std::isinf(v_descale)))
+    return fail(FA_ERR_INVALID_ARG, "fa_fwd_fp8: descale factors must be finite and > 0");
+  const int in_align = fp8 ? 16 : 8;  // elements per 16 bytes of input
   if (!q || !k || !v || !out) return fail(FA_ERR_INVALID_ARG, "fa_fwd: q, k, v and out must be non-NULL");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return fail(FA_ERR_INVALID_ARG, "fa_fwd: q, k, v and out must be 16-byte aligned");
@@ -242,8 +255,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
   const int64_t* vs = v_strides ? v_strides : dk;
   const int64_t* os = o_strides ? o_strides : dq;
   for (int i = varlen ? 1 : 0; i < 3; ++i)
-    if (qs[i] <= 0 || ks[i] <= 0 || vs[i] <= 0 || os[i] <= 0 || qs[i] % 8 || ks[i] % 8 || vs[i] % 8 || os[i] % 8)
-      return fail(FA_ERR_INVALID_ARG, "fa_fwd: strides must be positive multiples of 8 elements");
+    if (qs[i] <= 0 || ks[i] <= 0 || vs[i] <= 0 || os[i] <= 0 || qs[i] % in_align ||
+        ks[i] % in_align || vs[i] % in_align || os[i] % 8)
+      return fail(FA_ERR_INVALID_ARG, "fa_fwd: strides must be positive multiples of 16 bytes");
   const int rows_q = varlen ? max_seqlen_q : seqlen_q;
   if (batch == 0 || rows_q == 0) return FA_OK;  // nothing to compute
   const int n_tiles = (rows_q + 127) / 128;
@@ -254,15 +268,17 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
   if ((rc = device_state(nullptr, &status, nullptr)) != FA_OK) return rc;
 
   CUtensorMap tq, tk, tv;
-  const uint32_t box[4] = {64, 128, 1, 1};
+  // one 128-byte swizzle atom per row of the box: 64 16-bit or 128 8-bit elements
+  const uint32_t box[4] = {fp8 ? 128u : 64u, 128, 1, 1};
+  const uint64_t eb = fp8 ? 1 : 2;  // bytes per input element
   const uint64_t nb = varlen ? 1 : static_cast<uint64_t>(batch);
   {
     const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(std::max(seqlen_q, 1)),
                               static_cast<uint64_t>(H), nb};
-    const uint64_t st[3] = {static_cast<uint64_t>(qs[1]) * 2, static_cast<uint64_t>(qs[2]) * 2,
-                            varlen ? static_cast<uint64_t>(qs[1]) * 2 * std::max(seqlen_q, 1)
-                                   : static_cast<uint64_t>(qs[0]) * 2};
-    if ((rc = encode_4d(&tq, q, dims, st, box, "q")) != FA_OK) return rc;
+    const uint64_t st[3] = {static_cast<uint64_t>(qs[1]) * eb, static_cast<uint64_t>(qs[2]) * eb,
+                            varlen ? static_cast<uint64_t>(qs[1]) * eb * std::max(seqlen_q, 1)
+                                   : static_cast<uint64_t>(qs[0]) * eb};
+    if ((rc = encode_4d(&tq, q, dims, st, box, "q", fp8)) != FA_OK) return rc;
   }
   const int64_t* kvs[2] = {ks, vs};
   const void* kvp[2] = {k, v};
@@ -270,10 +286,11 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
   for (int t = 0; t < 2; ++t) {
     const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(std::max(seqlen_k, 1)),
                               static_cast<uint64_t>(Hkv), nb};
-    const uint64_t st[3] = {static_cast<uint64_t>(kvs[t][1]) * 2, static_cast<uint64_t>(kvs[t][2]) * 2,
-                            varlen ? static_cast<uint64_t>(kvs[t][1]) * 2 * std::max(seqlen_k, 1)
-                                   : static_cast<uint64_t>(kvs[t][0]) * 2};
-    if ((rc = encode_4d(kvm[t], kvp[t], dims, st, box, t == 0 ? "k" : "v")) != FA_OK) return rc;
+    const uint64_t st[3] = {static_cast<uint64_t>(kvs[t][1]) * eb, static_cast<uint64_t>(kvs[t][2]) * eb,
+                            varlen ? static_cast<uint64_t>(kvs[t][1]) * eb * std::max(seqlen_k, 1)
+                                   : static_cast<uint64_t>(kvs[t][0]) * eb};
+    if ((rc = encode_4d(kvm[t], kvp[t], dims, st, box, t == 0 ? "k" : "v", fp8)) != FA_OK)
+      return rc;
   }
 
   fa::FwdParams p{};
@@ -289,7 +306,10 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
   p.H = H;
   p.G = H / Hkv;
   p.total_q = seqlen_q;
-  fill_score_params(scale, softcap, &p.scale_log2, &p.softcap_log2, &p.tanh_k);
+  // 8-bit inputs: the scores carry q_descale * k_descale, folded into the scale
+  fill_score_params(fp8 ? scale * q_descale * k_descale : scale, softcap, &p.scale_log2,
+                    &p.softcap_log2, &p.tanh_k);
+  p.v_descale = fp8 ? v_descale : 1.f;
   p.alibi = alibi_slopes;
   p.causal = causal ? 1 : 0;
   p.wl = window_left;
@@ -298,11 +318,41 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
   p.status = status;
   p.timeout_ns = timeout_ns();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (dtype == FA_BF16)
+  cudaError_t e = fp8 ? fa::launch_fwd_fp8(tq, tk, tv, p, d, batch, rows_q, st)
+                  : (dtype == FA_BF16)
                       ? fa::launch_fwd_bf16(tq, tk, tv, p, d, batch, rows_q, st)
                       : fa::launch_fwd_f16(tq, tk, tv, p, d, batch, rows_q, st);
   if (e != cudaSuccess) return cuda_fail(e, "fa_fwd launch");
   return FA_OK;
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int dtype,
+           int batch, int seqlen_q, int seqlen_k, int num_heads, int num_heads_k, int head_dim,
+           const int64_t* q_strides, const int64_t* k_strides, const int64_t* v_strides,
+           const int64_t* o_strides, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+           int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal, int window_left,
+           int window_right, float softcap, const float* alibi_slopes, void* stream) {
+  g_err.clear();
+  return fwd_impl(q, k, v, out, lse, dtype, batch, seqlen_q, seqlen_k, num_heads, num_heads_k,
+                  head_dim, q_strides, k_strides, v_strides, o_strides, cu_seqlens_q,
+                  cu_seqlens_k, max_seqlen_q, max_seqlen_k, softmax_scale, causal, window_left,
+                  window_right, softcap, alibi_slopes, stream, false, 1.f, 1.f, 1.f);
+}
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse,
+               float q_descale, float k_descale, float v_descale, int batch, int seqlen_q,
+               int seqlen_k, int num_heads, int num_heads_k, int head_dim,
+               const int64_t* q_strides, const int64_t* k_strides, const int64_t* v_strides,
+               const int64_t* o_strides, const int32_t* cu_seqlens_q,
+               const int32_t* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k,
+               float softmax_scale, int causal, int window_left, int window_right,
+               float softcap, const float* alibi_slopes, void* stream) {
+  g_err.clear();
+  return fwd_impl(q, k, v, out, lse, FA_BF16, batch, seqlen_q, seqlen_k, num_heads, num_heads_k,
+                  head_dim, q_strides, k_strides, v_strides, o_strides, cu_seqlens_q,
+                  cu_seqlens_k, max_seqlen_q, max_seqlen_k, softmax_scale, causal, window_left,
+                  window_right, softcap, alibi_slopes, stream, true, q_descale, k_descale,
+                  v_descale);
 }
 
 // Query rows per KV head above which fa_fwd_kvcache runs the tensor-core prefill

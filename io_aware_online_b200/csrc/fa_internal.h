@@ -24,6 +24,7 @@ struct FwdParams {
   const float* alibi;              // [H] or NULL
   int causal, wl, wr;              // mask flags; -1 = unbounded window side
   int tile_major;                  // grid x = query tiles (no mask: equal work per tile)
+  float v_descale;                 // 8-bit inputs: O is multiplied by it (1 otherwise)
   // KV-cache mode (fa_fwd_kvcache with many query rows): K/V come from a paged pool
   // [num_blocks, page, Hkv, D] through block_table, or from a contiguous cache
   // [B, Sk, Hkv, D], in 64-row boxes; sequence b attends cache_seqlens[b] + k_add keys

@@ -47,15 +47,21 @@ constexpr uint32_t kSoftmaxRegs = 200;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
+// 8-bit P: the running max is kept exact (any growth rescales O) and P is taken
+// against max - 8, so P lies in (0, 256] (E4M3 tops out at 448) and values down to
+// 2^-17 of the row's largest stay in E4M3's normal range instead of underflowing.
+constexpr float kP8Offset = 8.0f;
 
 // T query tiles per CTA (1 or 2).  With T = 2 one CTA fills an SM (512 TMEM
 // columns, 12 warps); with T = 1 two CTAs share an SM (256 columns and 8 warps
 // each) and, being independent, drift out of phase, so that one CTA's
 // exponentials overlap the other's loads and reductions.
-template <int D, int T>
+// E = bytes per input element: 2 (fp16 / bf16) or 1 (E4M3, D = 128 only).
+template <int D, int T, int E = 2>
 struct FwdCfg {
   static_assert(T == 1 || T == 2, "one or two query tiles per CTA");
-  static_assert(T == 2 || D == 64, "one tile per CTA is laid out for D = 64 only");
+  static_assert(T == 2 || (D == 64 && E == 2), "one tile per CTA is laid out for 16-bit D = 64 only");
+  static_assert(E == 2 || D == 128, "8-bit inputs are laid out for D = 128 only");
   static constexpr int kThreads = (4 * T + 4) * 32;   // softmax warpgroups + one more
   static constexpr int kMinBlocks = 3 - T;             // CTAs per SM
   // registers a thread launches with, and what the non-softmax warpgroup keeps:
@@ -64,9 +70,10 @@ struct FwdCfg {
   static constexpr uint32_t kOtherRegs = (T == 2) ? 104 : 56;
   static_assert(T * 128 * kSoftmaxRegs + 128 * kOtherRegs == kThreads * kLaunchRegs,
                 "register re-split must add up to the launch registers");
-  static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms per row
-  static constexpr int kStages = (D == 128) ? 2 : (T == 2 ? 4 : 2);  // K and V ring depth
-  static constexpr int kTileBytes = 128 * D * 2;      // Q tile, K block or V block
+  static constexpr int kChunks = D * E / 128;         // 128-byte swizzle atoms per row
+  static constexpr int kChunkElems = 128 / E;         // elements per atom row
+  static constexpr int kStages = (D * E == 256) ? 2 : (T == 2 ? 4 : 2);  // K and V ring depth
+  static constexpr int kTileBytes = 128 * D * E;      // Q tile, K block or V block
   static constexpr int kChunkBytes = 128 * 128;       // 128 rows x 128 bytes
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + T * kTileBytes;
@@ -105,32 +112,48 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint6
 // S_t = Q_t K^T into tensor memory: K-major A (Q tile) and B (K block); a step of
 // 16 along the head dim is 32 bytes inside a 128-byte swizzle atom, the next atom
 // lies 16 KiB further.
-template <int D>
+// With 8-bit inputs (E = 1) a step is 32 elements, still 32 bytes, through
+// tcgen05.mma kind::f8f6f4.
+template <int D, int E = 2>
 __device__ __forceinline__ void fwd_issue_qk(uint32_t d_tmem, uint64_t a0, uint64_t b0,
                                              uint32_t idesc) {
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
+  for (int kk = 0; kk < D * E / 32; ++kk) {
     const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
-    mma_ss(d_tmem, desc_advance(a0, o), desc_advance(b0, o), idesc, kk > 0 ? 1u : 0u);
+    if constexpr (E == 2)
+      mma_ss(d_tmem, desc_advance(a0, o), desc_advance(b0, o), idesc, kk > 0 ? 1u : 0u);
+    else
+      mma_ss_f8(d_tmem, desc_advance(a0, o), desc_advance(b0, o), idesc, kk > 0 ? 1u : 0u);
   }
 }
 
 // O_t (+)= P_t V: A = P from tensor memory (8 columns hold 16 keys), B = V block,
 // MN-major (16 keys = 16 rows = 2 KiB; head-dim atoms 16 KiB apart).
-template <int D>
+// With 8-bit P and V a step is 32 keys: 8 columns of four E4M3 values, 4 KiB of V.
+template <int D, int E = 2>
 __device__ __forceinline__ void fwd_issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
                                              uint32_t idesc, bool acc) {
 #pragma unroll
-  for (int kk = 0; kk < kBN / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + kk * 8, desc_advance(b0, kk * 2048), idesc,
-           (acc || kk > 0) ? 1u : 0u);
+  for (int kk = 0; kk < kBN * E / 32; ++kk) {
+    if constexpr (E == 2)
+      mma_ts(d_tmem, a_tmem + kk * 8, desc_advance(b0, kk * 2048), idesc,
+             (acc || kk > 0) ? 1u : 0u);
+    else
+      mma_ts_f8(d_tmem, a_tmem + kk * 8, desc_advance(b0, kk * 4096), idesc,
+                (acc || kk > 0) ? 1u : 0u);
+  }
 }
 
-template <int D, int T, bool BF16, bool SOFTCAP, bool ALIBI, int EMU>
-__global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBlocks)
+// FP8: E4M3 Q, K, V (both products on kind::f8f6f4, P rounded to E4M3), bf16 output
+// (BF16 must then be true).
+template <int D, int T, bool BF16, bool SOFTCAP, bool ALIBI, int EMU, bool FP8 = false>
+__global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
+                                  FwdCfg<D, T, FP8 ? 1 : 2>::kMinBlocks)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using Cfg = FwdCfg<D, T>;
+  static_assert(!FP8 || BF16, "8-bit inputs write a bf16 output");
+  constexpr int E = FP8 ? 1 : 2;
+  using Cfg = FwdCfg<D, T, E>;
   constexpr int ST = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -242,7 +265,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
       mbar_arrive_expect_tx(q_full, T * Cfg::kTileBytes);
       for (int t = 0; t < T; ++t)
         for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_4d(sQ + t * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmQ, q_full, c * 64,
+          tma_load_4d(sQ + t * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmQ, q_full, c * Cfg::kChunkElems,
                       qrow + t * kBM, h, b_coord);
       int last_k[ST], last_v[ST];
       for (int s = 0; s < ST; ++s) last_k[s] = last_v[s] = -1;
@@ -255,13 +278,13 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
           mbar_arrive_expect_tx(k_full + s, Cfg::kTileBytes);
           for (int c = 0; c < Cfg::kChunks; ++c)
             tma_load_4d(sK + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmK, k_full + s,
-                        c * 64, krow + j * kBN, hk, b_coord);
+                        c * Cfg::kChunkElems, krow + j * kBN, hk, b_coord);
           last_k[s] = ph;
           if (!wait_bounded(v_empty + s, ph ^ 1, w)) break;
           mbar_arrive_expect_tx(v_full + s, Cfg::kTileBytes);
           for (int c = 0; c < Cfg::kChunks; ++c)
             tma_load_4d(sV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmV, v_full + s,
-                        c * 64, krow + j * kBN, hk, b_coord);
+                        c * Cfg::kChunkElems, krow + j * kBN, hk, b_coord);
           last_v[s] = ph;
         } else {
           // KV cache: the block's two 64-key halves, each inside one page (page_size
@@ -291,14 +314,14 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
           for (int hh = 0; hh < nh; ++hh)
             for (int c = 0; c < Cfg::kChunks; ++c)
               tma_load_4d(sK + s * Cfg::kTileBytes + c * Cfg::kChunkBytes + hh * 64 * 128, &tmK,
-                          k_full + s, c * 64, row[hh], hk, blk[hh]);
+                          k_full + s, c * Cfg::kChunkElems, row[hh], hk, blk[hh]);
           last_k[s] = ph;
           if (!wait_bounded(v_empty + s, ph ^ 1, w)) break;
           mbar_arrive_expect_tx(v_full + s, nh * kHalfBytes);
           for (int hh = 0; hh < nh; ++hh)
             for (int c = 0; c < Cfg::kChunks; ++c)
               tma_load_4d(sV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes + hh * 64 * 128, &tmV,
-                          v_full + s, c * 64, row[hh], hk, blk[hh]);
+                          v_full + s, c * Cfg::kChunkElems, row[hh], hk, blk[hh]);
           last_v[s] = ph;
         }
       }
@@ -316,17 +339,17 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
     // One thread alternates the tiles, PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so
     // one tile's softmax overlaps the other tile's products.
     if (lane == 0 && n_blk > 0) {
-      constexpr uint32_t idesc_qk = f16_idesc(BF16, kBM, kBN, false, false);
-      constexpr uint32_t idesc_pv = f16_idesc(BF16, kBM, D, false, true);
+      constexpr uint32_t idesc_qk = f16_idesc(BF16 && !FP8, kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = f16_idesc(BF16 && !FP8, kBM, D, false, true);
       const uint64_t dQ0 = sw128_desc(smem_u32(sQ), 16, 1024);
       const uint64_t dQ1 = desc_advance(dQ0, Cfg::kTileBytes);
       const uint64_t dK = sw128_desc(smem_u32(sK), 16, 1024);
       const uint64_t dV = sw128_desc(smem_u32(sV), Cfg::kChunkBytes, 1024);
 #define FA_QK(T, S)                                                                    \
-  fwd_issue_qk<D>(tbase + (T) * kBM, (T) ? dQ1 : dQ0,                                    \
+  fwd_issue_qk<D, E>(tbase + (T) * kBM, (T) ? dQ1 : dQ0,                                    \
                   desc_advance(dK, (S) * Cfg::kTileBytes), idesc_qk)
 #define FA_PV(T, S, ACC)                                                               \
-  fwd_issue_pv<D>(tbase + Cfg::kOCol + (T) * D, tbase + Cfg::kPCol + (T) * Cfg::kPStride, \
+  fwd_issue_pv<D, E>(tbase + Cfg::kOCol + (T) * D, tbase + Cfg::kPCol + (T) * Cfg::kPStride, \
                   desc_advance(dV, (S) * Cfg::kTileBytes), idesc_pv, ACC)
       bool ok = wait_bounded(q_full, 0, w) && wait_bounded(k_full, 0, w);
       if (ok) {
@@ -380,17 +403,17 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
     // ======================================================== MMA issuers (D = 64)
     const int t = warp - Cfg::kIssuerWarp;  // this issuer's query tile
     if (lane == 0 && n_blk > 0) {
-      constexpr uint32_t idesc_qk = f16_idesc(BF16, kBM, kBN, false, false);
-      constexpr uint32_t idesc_pv = f16_idesc(BF16, kBM, D, false, true);
+      constexpr uint32_t idesc_qk = f16_idesc(BF16 && !FP8, kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = f16_idesc(BF16 && !FP8, kBM, D, false, true);
       const uint32_t tS = tbase + t * kBM;
       const uint32_t tP = tbase + Cfg::kPCol + t * Cfg::kPStride;
       const uint32_t tO = tbase + Cfg::kOCol + t * D;
       const uint64_t dQ = desc_advance(sw128_desc(smem_u32(sQ), 16, 1024), t * Cfg::kTileBytes);
       const uint64_t dK = sw128_desc(smem_u32(sK), 16, 1024);               // K-major
       const uint64_t dV = sw128_desc(smem_u32(sV), Cfg::kChunkBytes, 1024); // MN-major
-#define FA_QK(S) fwd_issue_qk<D>(tS, dQ, desc_advance(dK, (S) * Cfg::kTileBytes), idesc_qk)
+#define FA_QK(S) fwd_issue_qk<D, E>(tS, dQ, desc_advance(dK, (S) * Cfg::kTileBytes), idesc_qk)
 #define FA_PV(S, ACC) \
-  fwd_issue_pv<D>(tO, tP, desc_advance(dV, (S) * Cfg::kTileBytes), idesc_pv, ACC)
+  fwd_issue_pv<D, E>(tO, tP, desc_advance(dV, (S) * Cfg::kTileBytes), idesc_pv, ACC)
       bool ok = wait_bounded(q_full, 0, w) && wait_bounded(k_full, 0, w);
       if (ok) {
         tc_fence_after();
@@ -509,14 +532,15 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
       // (rows whose max did not move recompute the same values).  The raw scores
       // stay in registers until that check.  Warps with a row that has not met an
       // allowed key yet (running max -inf) take the max-first order.
-      const bool spec = !Cfg::kSepP && __all_sync(0xffffffffu, m_use != -INFINITY);
+      const bool spec = !Cfg::kSepP && !FP8 && __all_sync(0xffffffffu, m_use != -INFINITY);
+      constexpr float kThreshold = FP8 ? 0.f : kRescaleThreshold;
       bool need = false;
       float alpha = 1.f;
       auto update_max = [&](float m_blk) {
         const float m_new = fmaxf(m_use, m_blk);
         if (m_use == -INFINITY) {
           m_use = m_new;  // nothing accumulated yet: O is zero
-        } else if (m_new > m_use + kRescaleThreshold) {
+        } else if (m_new > m_use + kThreshold) {
           need = true;
           alpha = ex2(m_use - m_new);
           m_use = m_new;
@@ -542,8 +566,9 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
       uint32_t pk[Cfg::kSepP ? kBN / 2 : 16];
       auto exps = [&](auto with_max) {
         constexpr bool kMax = decltype(with_max)::value;
-        const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+        const float neg_m = (m_use == -INFINITY) ? 0.f : (FP8 ? kP8Offset : 0.f) - m_use;
         const float2 f2 = make_float2(factor, factor), nm2 = make_float2(neg_m, neg_m);
+        float2 prev = make_float2(0.f, 0.f);
 #pragma unroll
         for (int q4 = 0; q4 < kBN / 32; ++q4) {
           lsum[q4] = make_float2(0.f, 0.f);
@@ -564,14 +589,24 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
               pp = exp2_fma2(arg);
             else
               pp = make_float2(ex2(arg.x), ex2(arg.y));
-            const int pi = Cfg::kSepP ? q4 * 16 + e : e;
-            pk[pi] = pack2<BF16>(pp.x, pp.y);
             lsum[q4] = add2(lsum[q4], pp);
-            // bf16 P is rounded by up to 2^-9: sum the rounded values the PV product
-            // uses, so that O / lr is an exact convex combination of V rows
-            if constexpr (BF16) lrnd[q4] = add2(lrnd[q4], unpack2<true>(pk[pi]));
+            if constexpr (FP8) {  // four E4M3 values per column, consecutive keys
+              if (e % 2 == 0)
+                prev = pp;
+              else
+                pk[e / 2] = pack4_e4m3(prev.x, prev.y, pp.x, pp.y);
+            } else {
+              const int pi = Cfg::kSepP ? q4 * 16 + e : e;
+              pk[pi] = pack2<BF16>(pp.x, pp.y);
+              // bf16 P is rounded by up to 2^-9: sum the rounded values the PV
+              // product uses, so that O / lr is an exact convex combination of V rows
+              if constexpr (BF16) lrnd[q4] = add2(lrnd[q4], unpack2<true>(pk[pi]));
+            }
           }
-          if constexpr (!Cfg::kSepP) tmem_st16(tP + q4 * 16, pk);
+          if constexpr (FP8)
+            tmem_st8(tP + q4 * 8, pk);
+          else if constexpr (!Cfg::kSepP)
+            tmem_st16(tP + q4 * 16, pk);
         }
       };
       if (spec) {
@@ -599,7 +634,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
       {
         float2 a = add2(add2(lsum[0], lsum[1]), add2(lsum[2], lsum[3]));
         l += a.x + a.y;
-        if constexpr (BF16) a = add2(add2(lrnd[0], lrnd[1]), add2(lrnd[2], lrnd[3]));
+        if constexpr (BF16 && !FP8) a = add2(add2(lrnd[0], lrnd[1]), add2(lrnd[2], lrnd[3]));
         lr += a.x + a.y;
       }
       // O_t rescale (after the score row is dead: lower register peak); it only
@@ -651,7 +686,8 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
       // a row with no allowed key keeps m = -inf (its sum may hold clamped
       // polynomial exponentials of -inf, each <= 2^-126): O = 0, LSE = -inf
       const bool dead = (m_use == -INFINITY) || !(lr > 0.f);
-      const float inv = dead ? 0.f : 1.f / lr;
+      // 8-bit inputs: O carries V's descale factor (Q's and K's sit in the scale)
+      const float inv = dead ? 0.f : (FP8 ? p.v_descale : 1.f) / lr;
       uint8_t* orow = nullptr;
       if (row_ok) {
         const int64_t ro = varlen ? static_cast<int64_t>(q0 + i) * p.o_ss
@@ -681,7 +717,8 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, FwdCfg<D, T>::kMinBloc
         }
       }
       if (row_ok && p.lse != nullptr) {
-        const float lse = dead ? -INFINITY : (m_use + __log2f(l)) * kLn2;
+        const float lse =
+            dead ? -INFINITY : (m_use - (FP8 ? kP8Offset : 0.f) + __log2f(l)) * kLn2;
         const int64_t li = varlen ? static_cast<int64_t>(h) * p.total_q + q0 + i
                                   : (static_cast<int64_t>(b) * p.H + h) * p.Sq + i;
         p.lse[li] = lse;

@@ -8,11 +8,11 @@
 
 namespace fa {
 
-template <int D, int T, bool BF16, bool SOFTCAP, bool ALIBI, int EMU>
+template <int D, int T, bool BF16, bool SOFTCAP, bool ALIBI, int EMU, bool FP8 = false>
 cudaError_t launch_fwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int batch, int rows_q, cudaStream_t stream) {
-  using Cfg = FwdCfg<D, T>;
-  auto kern = fwd_kernel<D, T, BF16, SOFTCAP, ALIBI, EMU>;
+  using Cfg = FwdCfg<D, T, FP8 ? 1 : 2>;
+  auto kern = fwd_kernel<D, T, BF16, SOFTCAP, ALIBI, EMU, FP8>;
   constexpr int smem = Cfg::kSmemAlloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess && T == 1)  // room for two CTAs per SM

@@ -177,3 +177,15 @@ def test_fwd_kvcache_append_validation(lib):
 def test_selftest_limit_validation(lib):
     assert lib.fa_selftest_wait_timeout(0, None) == FA_ERR_INVALID_ARG
     assert lib.fa_selftest_wait_timeout(20000, None) == FA_ERR_INVALID_ARG
+
+
+def test_fp8_validation(lib):
+    def f8(**kw):
+        a = dict(qd=1.0, kd=1.0, vd=1.0, d=128)
+        a.update(kw)
+        return lib.fa_fwd_fp8(P, P, P, P, None, a["qd"], a["kd"], a["vd"], 1, 128, 128, 2, 2,
+                              a["d"], None, None, None, None, None, None, 0, 0,
+                              float("nan"), 0, -1, -1, 0.0, None, None)
+    assert f8(d=64) == FA_ERR_UNSUPPORTED
+    assert f8(qd=0.0) == FA_ERR_INVALID_ARG
+    assert f8(vd=float("inf")) == FA_ERR_INVALID_ARG
