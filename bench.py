@@ -326,6 +326,64 @@ def run_ours(args, rank, world, local):
 # and a whole 8192-token prompt written into an empty paged cache (append).
 CHUNKED = dict(B=4, cached=6144, chunk=2048, H=32, Hkv=8, d=128, dtype="bf16", page=256)
 APPEND = dict(B=4, S_new=8192, Hkv=8, d=128, dtype="bf16", page=256)
+# 8-bit forward (fa_fwd_fp8): the d=128 prefill point, E4M3 inputs cast from N(0,1)
+FP8 = dict(B=4, S=8192, H=32, Hkv=32, d=128, dtype="e4m3", causal=True)
+
+
+def run_fp8(args, rank, world, local):
+    """--only fp8: time fa_fwd_fp8 on the d=128 causal prefill workload."""
+    import io_aware_online_b200 as fa
+    from io_aware_online_b200 import build as fa_build
+    fa_build.build()
+    fa.load()
+    dev = torch.device("cuda", local)
+    hbm_peak, tflops_peak, peak_src = load_peaks()
+    fp8_peak = 2.0 * tflops_peak       # dense e4m3 vs bf16: 4.5 / 2.25 PFLOP/s nominal
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    c = FP8
+    gen = torch.Generator(device=dev).manual_seed(3100 + rank)
+    shape_q = (c["B"], c["S"], c["H"], c["d"])
+    shape_k = (c["B"], c["S"], c["Hkv"], c["d"])
+    q = torch.randn(shape_q, generator=gen, device=dev).to(torch.float8_e4m3fn)
+    k = torch.randn(shape_k, generator=gen, device=dev).to(torch.float8_e4m3fn)
+    v = torch.randn(shape_k, generator=gen, device=dev).to(torch.float8_e4m3fn)
+    out = torch.empty(shape_q, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((c["B"], c["H"], c["S"]), dtype=torch.float32, device=dev)
+    work = 4.0 * c["d"] * c["B"] * c["H"] * causal_pairs(c["S"], c["S"])
+
+    def call():
+        fa.fa_fwd_fp8(q, k, v, out=out, lse=lse, causal=True, stream=stream)
+    for _ in range(args.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with Clocks(dev.index if dev.index is not None else 0) as clk:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world)
+    achieved = work / (ms * 1e-3) / 1e12
+    return {"metric": "attn fwd TFLOPS, E4M3 inputs (causal prefill)", "value": round(achieved * world, 2),
+            "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3 (bf16 out)", "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": "fp8", **c, "l2": "flushed between steps (256 MiB write, "
+                       "untimed)", "parallelism": f"dp{world} (independent replicas)"},
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": fp8_peak,
+                         "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
+                         "traffic": None,
+                         "kernel": "fwd_kernel<128, 2 tiles, e4m3, causal> (kind::f8f6f4)",
+                         "peak_source": f"{peak_src} bf16 burst x 2 (nominal e4m3/bf16 ratio)"},
+            "gpu_launches": K, "clocks": clk.summary()}
 
 
 def run_cache_rows(args, rank, world, local):
@@ -500,7 +558,7 @@ def main():
     ap.add_argument("--num-splits", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "chunked", "append"],
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "chunked", "append", "fp8"],
                     default="all",
                     help="time one part of the step (profiling / sweeps), or one of the "
                          "cache-update rows on its own workload (chunked, append)")
@@ -519,8 +577,8 @@ def main():
             if rank == 0:
                 print(json.dumps(run_reference(args, rank, world)), flush=True)
             return
-        if args.only in ("chunked", "append"):
-            res = run_cache_rows(args, rank, world, local)
+        if args.only in ("chunked", "append", "fp8"):
+            res = (run_fp8 if args.only == "fp8" else run_cache_rows)(args, rank, world, local)
             if rank == 0:
                 print(json.dumps(res), flush=True)
             return
