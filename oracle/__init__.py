@@ -18,6 +18,7 @@ attention_paged(q, kpool, vpool, block_table, cache_seqlens, ...)
 combine(out_partial, lse_partial)          LSE-weighted combine of split partials
 append(kcache, vcache, k_new, v_new, cache_seqlens, block_table=None)
                                            KV-cache append (returns updated copies)
+attention_backward(q, k, v, do, ...)       gradients dq, dk, dv (backward.py, numpy fp64)
 """
 from __future__ import annotations
 
@@ -224,3 +225,6 @@ def append(kcache, vcache, k_new, v_new, cache_seqlens, block_table=None):
                 kc[b, x] = kn[b, t]
                 vc[b, x] = vn[b, t]
     return kc, vc
+
+
+from .backward import attention_backward  # noqa: E402,F401  (fp64 gradients; see backward.py)
