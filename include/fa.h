@@ -247,6 +247,39 @@ FA_API int fa_fwd_kvcache_append(const void *q, void *k_cache, void *v_cache, co
                                  void *stream);
 
 /*
+ * fa_bwd_workspace_size -- bytes of device scratch fa_bwd needs: batch *
+ * num_heads * seqlen_q fp32 values (D = rowsum(dO * O)), rounded up to 256.
+ */
+FA_API size_t fa_bwd_workspace_size(int batch, int seqlen_q, int num_heads);
+
+/*
+ * fa_bwd -- gradients of the dense attention forward (tag page "flash attention":
+ * the backward recomputes the attention matrix tile by tile from Q, K and the
+ * forward's softmax statistics instead of reading a stored one).
+ *
+ *   dout, q, out, dq: [batch, seqlen_q, num_heads, head_dim] contiguous, 16-bit
+ *   (dtype as for fa_fwd); k, v, dk, dv: [batch, seqlen_k, num_heads_k, head_dim]
+ *   contiguous; lse: fp32 [batch, num_heads, seqlen_q], the forward's LSE;
+ *   out: the forward's O.  The mask, scale, window and ALiBi arguments must be
+ *   those of the forward call; softcap must be 0 (its backward is not built:
+ *   FA_ERR_UNSUPPORTED).
+ * Computes, with P = exp(scale Q K^T + bias - LSE) on the allowed entries and
+ * D = rowsum(dout * out): dv = P^T dout, dS = P * (dout v^T - D),
+ * dq = scale dS k, dk = scale dS^T q; dk and dv sum over the query heads that
+ * share a KV head.  Deterministic (no atomics): one pass per key block for dk/dv,
+ * one per query block for dq.  P and dS are rounded to the input dtype before
+ * their products (fp32 accumulation).
+ * workspace: >= fa_bwd_workspace_size(batch, seqlen_q, num_heads) bytes, 16-byte
+ *   aligned; calls sharing it must be stream-ordered.
+ */
+FA_API int fa_bwd(const void *dout, const void *q, const void *k, const void *v,
+                  const void *out, const float *lse, void *dq, void *dk, void *dv, int dtype,
+                  int batch, int seqlen_q, int seqlen_k, int num_heads, int num_heads_k,
+                  int head_dim, float softmax_scale, int causal, int window_left,
+                  int window_right, float softcap, const float *alibi_slopes, void *workspace,
+                  size_t workspace_bytes, void *stream);
+
+/*
  * fa_selftest_wait_timeout -- a diagnostic of the bounded waits (the pages have no
  * counterpart): launches one CTA that waits, through the library's bounded wait, on
  * a barrier phase nothing ever completes.  After timeout_ms (1..10000) of GPU time

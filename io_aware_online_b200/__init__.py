@@ -91,6 +91,11 @@ def load():
     lib.fa_device_status.restype = i32
     lib.fa_set_wait_timeout_ms.argtypes = [i32]
     lib.fa_set_wait_timeout_ms.restype = i32
+    lib.fa_bwd_workspace_size.argtypes = [i32, i32, i32]
+    lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                           f32, i32, i32, i32, f32, vp, vp, ctypes.c_size_t, vp]
+    lib.fa_bwd.restype = i32
     lib.fa_selftest_wait_timeout.argtypes = [i32, vp]
     lib.fa_selftest_wait_timeout.restype = i32
     lib.fa_version.argtypes = []
@@ -355,3 +360,29 @@ def fa_selftest_wait_timeout(timeout_ms=20, stream=None):
     """Launch the bounded-wait self-test (include/fa.h): after timeout_ms the waiting
     CTA raises FA_DEV_WAIT_TIMEOUT in the device status word and exits."""
     _check(load().fa_selftest_wait_timeout(int(timeout_ms), _stream(stream)))
+
+
+def fa_bwd(dout, q, k, v, out, lse, *, softmax_scale=None, causal=False, window_size=(-1, -1),
+           alibi_slopes=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of the dense forward for output gradient dout; q, out,
+    dout [B, Sq, H, d], k, v [B, Sk, Hkv, d] contiguous, lse [B, H, Sq] from fa_fwd
+    (same mask arguments as the forward call)."""
+    lib = load()
+    dt = _dtype(q)
+    B, sq, H, d = q.shape
+    sk, Hkv = k.shape[1], k.shape[2]
+    for t in (dout, q, k, v, out, lse):
+        if not t.is_contiguous():
+            raise ValueError("fa_bwd takes contiguous tensors")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = lib.fa_bwd_workspace_size(B, sq, H)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.fa_bwd(_ptr(dout), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dq),
+                      _ptr(dk), _ptr(dv), dt, B, sq, sk, H, Hkv, d, _scale(softmax_scale),
+                      int(bool(causal)), int(window_size[0]), int(window_size[1]), 0.0,
+                      _ptr(alibi_slopes), _ptr(workspace), ws_bytes, _stream(stream)))
+    return dq, dk, dv

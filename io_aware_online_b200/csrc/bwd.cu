@@ -1,0 +1,612 @@
+// bwd.cu -- attention backward for sm_100a: dQ, dK, dV of
+// O = softmax(mask(scale Q K^T) + ALiBi) V, recomputing the attention matrix
+// tile by tile from Q, K and the forward's LSE instead of storing it (tag page
+// "flash attention": the backward recomputes S and P in on-chip memory).
+//
+// With P = exp(S - LSE), dP = dO V^T, D = rowsum(dO * O) and dS = P * (dP - D):
+//   dV = P^T dO,  dK = scale * dS^T Q,  dQ = scale * dS K.
+// Three kernels, all deterministic (no atomics):
+//   bwd_dot_kernel   D for every query row (one warp per row).
+//   bwd_dkdv_kernel  one CTA per (128-key block, KV head): K_j and V_j stay in
+//                    shared memory while the query blocks (of every query head
+//                    reading this KV head) stream past; per block
+//                      S^T = K_j Q_i^T, dP^T = V_j dO_i^T   (tcgen05, SS)
+//                      P^T, dS^T in registers -> 16-bit in tensor memory
+//                      dV += P^T dO_i, dK += dS^T Q_i        (tcgen05, TS)
+//                    with dV and dK accumulated in tensor memory.
+//   bwd_dq_kernel    one CTA per (128-query block, head): Q_i and dO_i stay in
+//                    shared memory while the key blocks stream past; per block
+//                      S = Q_i K_j^T, dP = dO_i V_j^T, dS -> 16-bit,
+//                      dQ += dS K_j                           (tcgen05)
+// Roles per CTA (256 threads): warps 0-3 compute (thread r owns tensor-memory
+// lane r: a key row in dK/dV, a query row in dQ), warp 4 TMA producer, warp 5
+// MMA issuer (one elected thread; it also allocates tensor memory), warps 6-7
+// idle.  Tensor memory: S [0,128), dP [128,256), accumulators from 256; P and dS
+// are written as 16-bit pairs over the first 64 columns of S and dP, which the
+// thread has already read.  Every wait is bounded.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+
+#include "fa_internal.h"
+#include "fwd_kernel.cuh"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kBwdThreads = 256;
+constexpr float kBwdLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms per row
+  static constexpr int kTileBytes = 128 * D * 2;      // one 128-row tile
+  static constexpr int kChunkBytes = 128 * 128;
+  static constexpr int kFixA = 0;                     // K_j (dK/dV) or Q_i (dQ)
+  static constexpr int kFixB = kTileBytes;            // V_j (dK/dV) or dO_i (dQ)
+  static constexpr int kStage = 2 * kTileBytes;       // 2 stages x {A, B} streamed tiles
+  static constexpr int kStat = kStage + 4 * kTileBytes;  // [2 slots][2][128] fp32
+  static constexpr int kBarOff = kStat + 2 * 2 * 128 * 4;
+  // fix_full, full[2], empty[2], s_full, p_full, stat[2], done, drain
+  static constexpr int kNumBars = 11;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16;
+  // room to align the base to 1 KiB; at least 116 KiB, so that one CTA fills an SM
+  // (each takes all 512 tensor-memory columns; a second one would wait in its
+  // allocation for the first to finish)
+  static constexpr int kSmemAlloc =
+      (kSmemBytes + 1024 > 116 * 1024) ? kSmemBytes + 1024 : 116 * 1024;
+  static constexpr int kTmemCols = 512;                 // S 128 + dP 128 + up to 2 x D
+};
+
+// Key j allowed for query i (bottom-right alignment, off = Sk - Sq).
+struct MaskGeo {
+  int off, Sk, Sq, wl, right;
+  bool has_left, has_right;
+  __device__ __forceinline__ bool allowed(int i, int j) const {
+    if (i >= Sq || j >= Sk) return false;
+    const int c = i + off;
+    if (has_right && j > c + right) return false;
+    if (has_left && j < c - wl) return false;
+    return true;
+  }
+};
+
+__device__ __forceinline__ MaskGeo mask_geo(const BwdParams& p) {
+  MaskGeo g;
+  g.off = p.Sk - p.Sq;
+  g.Sk = p.Sk;
+  g.Sq = p.Sq;
+  g.wl = p.wl;
+  g.has_left = p.wl >= 0;
+  g.has_right = p.causal || p.wr >= 0;
+  g.right = p.causal ? 0 : p.wr;
+  return g;
+}
+
+__device__ __forceinline__ bool wait_drain_bwd(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+  return true;
+}
+
+// D[b, h, i] = sum_c dO[b, i, h, c] * O[b, i, h, c], fp32; one warp per row.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) bwd_dot_kernel(const BwdParams p) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + threadIdx.x / 32;  // (b, i, h)
+  const int lane = threadIdx.x % 32;
+  if (row >= static_cast<int64_t>(p.B) * p.Sq * p.H) return;
+  constexpr int kPer = D / 32;  // elements per lane: 2 or 4
+  const uint16_t* o = static_cast<const uint16_t*>(p.out) + row * D + lane * kPer;
+  const uint16_t* g = static_cast<const uint16_t*>(p.dout) + row * D + lane * kPer;
+  float acc = 0.f;
+#pragma unroll
+  for (int e = 0; e < kPer; e += 2) {
+    const float2 a = unpack2<BF16>(*reinterpret_cast<const uint32_t*>(o + e));
+    const float2 c = unpack2<BF16>(*reinterpret_cast<const uint32_t*>(g + e));
+    acc = fmaf(a.x, c.x, fmaf(a.y, c.y, acc));
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if (lane == 0) {
+    const int h = static_cast<int>(row % p.H);
+    const int64_t bi = row / p.H;  // b * Sq + i
+    const int i = static_cast<int>(bi % p.Sq);
+    const int b = static_cast<int>(bi / p.Sq);
+    p.dvec[(static_cast<int64_t>(b) * p.H + h) * p.Sq + i] = acc;
+  }
+}
+
+// One CTA per (128-key block kb, KV head hk, batch b).
+template <int D, bool BF16, bool ALIBI>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const BwdParams p) {
+  using Cfg = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int k0 = blockIdx.x * 128;
+  const int hk = blockIdx.y;
+  const int b = blockIdx.z;
+  const MaskGeo mg = mask_geo(p);
+  // query rows that see some key of [k0, k1)
+  const int k1 = min(k0 + 128, p.Sk);
+  const int q_lo = mg.has_right ? max(0, k0 - mg.off - mg.right) : 0;
+  const int q_hi = mg.has_left ? min(p.Sq - 1, k1 - 1 - mg.off + mg.wl) : p.Sq - 1;
+  const int i_lo = q_lo / 128;
+  const int nqb = (q_hi >= q_lo && k0 < p.Sk) ? q_hi / 128 - i_lo + 1 : 0;
+  const int n_iter = p.G * nqb;  // iteration n: head hk * G + n / nqb, query block i_lo + n % nqb
+
+  uint8_t* fixA = smem + Cfg::kFixA;  // K_j
+  uint8_t* fixB = smem + Cfg::kFixB;  // V_j
+  uint8_t* stage = smem + Cfg::kStage;  // slot s: Q_i at s * 2 tiles, dO_i after it
+  float* stat = reinterpret_cast<float*>(smem + Cfg::kStat);  // [slot][lse2 | D][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
+  uint64_t* fix_full = bars;
+  uint64_t* full = bars + 1;
+  uint64_t* empty = bars + 3;
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* statb = bars + 7;
+  uint64_t* done = bars + 9;
+  uint64_t* drain = bars + 10;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
+
+  if (warp == 4 && lane == 0) {
+    mbar_init(fix_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+      mbar_init(statb + s, 4);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_holder, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+  const WaitCtx w{abort_flag, p.status, p.timeout_ns};
+
+  if (warp == 4) {
+    // ======================================================== TMA producer
+    if (lane == 0 && n_iter > 0) {
+      tma_prefetch_map(&tmQ);
+      tma_prefetch_map(&tmK);
+      tma_prefetch_map(&tmV);
+      tma_prefetch_map(&tmDO);
+      mbar_arrive_expect_tx(fix_full, 2 * Cfg::kTileBytes);
+      for (int c = 0; c < Cfg::kChunks; ++c) {
+        tma_load_4d(fixA + c * Cfg::kChunkBytes, &tmK, fix_full, c * 64, k0, hk, b);
+        tma_load_4d(fixB + c * Cfg::kChunkBytes, &tmV, fix_full, c * 64, k0, hk, b);
+      }
+      int last[2] = {-1, -1};
+      for (int n = 0; n < n_iter; ++n) {
+        const int s = n & 1;
+        const uint32_t ph = (n >> 1) & 1;
+        const int h = hk * p.G + n / nqb;
+        const int qb = (i_lo + n % nqb) * 128;
+        if (!wait_bounded(empty + s, ph ^ 1, w)) break;
+        mbar_arrive_expect_tx(full + s, 2 * Cfg::kTileBytes);
+        uint8_t* st = stage + s * 2 * Cfg::kTileBytes;
+        for (int c = 0; c < Cfg::kChunks; ++c) {
+          tma_load_4d(st + c * Cfg::kChunkBytes, &tmQ, full + s, c * 64, qb, h, b);
+          tma_load_4d(st + Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmDO, full + s, c * 64, qb, h,
+                      b);
+        }
+        last[s] = ph;
+      }
+      if (*abort_flag) {  // let this CTA's own copies land before the smem goes away
+        wait_drain_bwd(fix_full, 0, p.timeout_ns);
+        for (int s = 0; s < 2; ++s)
+          if (last[s] >= 0) wait_drain_bwd(full + s, last[s], p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ======================================================== MMA issuer
+    if (lane == 0 && n_iter > 0) {
+      constexpr uint32_t idesc_s = f16_idesc(BF16, 128, 128, false, false);
+      constexpr uint32_t idesc_acc = f16_idesc(BF16, 128, D, false, true);
+      const uint64_t dKk = sw128_desc(smem_u32(fixA), 16, 1024);  // K-major operands
+      const uint64_t dVk = sw128_desc(smem_u32(fixB), 16, 1024);
+      bool ok = wait_bounded(fix_full, 0, w);
+      for (int n = 0; n < n_iter && ok; ++n) {
+        const int s = n & 1;
+        const uint32_t ph = (n >> 1) & 1;
+        if (!(ok = wait_bounded(full + s, ph, w))) break;
+        tc_fence_after();
+        const uint32_t sq = smem_u32(stage + s * 2 * Cfg::kTileBytes);
+        const uint32_t sdo = sq + Cfg::kTileBytes;
+        fwd_issue_qk<D>(tbase, dKk, sw128_desc(sq, 16, 1024), idesc_s);          // S^T
+        fwd_issue_qk<D>(tbase + 128, dVk, sw128_desc(sdo, 16, 1024), idesc_s);   // dP^T
+        tc_commit(s_full);
+        if (!(ok = wait_bounded(p_full, n & 1, w))) break;
+        tc_fence_after();
+        // B operands MN-major: rows are queries, the head dim contiguous
+        fwd_issue_pv<D>(tbase + 256, tbase, sw128_desc(sdo, Cfg::kChunkBytes, 1024), idesc_acc,
+                        n > 0);                                                   // dV
+        fwd_issue_pv<D>(tbase + 256 + D, tbase + 128, sw128_desc(sq, Cfg::kChunkBytes, 1024),
+                        idesc_acc, n > 0);                                        // dK
+        tc_commit(empty + s);
+      }
+      if (ok) tc_commit(done);
+      tc_commit(drain);
+      wait_drain_bwd(drain, 0, p.timeout_ns);  // own MMAs complete before teardown
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ======================================================== compute
+    const int r = threadIdx.x;  // key row within the block = TMEM lane
+    const int k = k0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    bool ok = true;
+    for (int n = 0; n < n_iter; ++n) {
+      const int s = n & 1;
+      const int h = hk * p.G + n / nqb;
+      const int qb = (i_lo + n % nqb) * 128;
+      const float slope2 = ALIBI ? p.alibi[h] * kBwdLog2e : 0.f;
+      // column statistics of this query block: thread r provides query qb + r
+      {
+        const int q = qb + r;
+        const int64_t idx = (static_cast<int64_t>(b) * p.H + h) * p.Sq + q;
+        float* slot = stat + s * 256;
+        slot[r] = (q < p.Sq) ? p.lse[idx] * kBwdLog2e : INFINITY;  // P = 0 past the end
+        slot[128 + r] = (q < p.Sq) ? p.dvec[idx] : 0.f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(statb + s);
+      }
+      ok = wait_bounded(statb + s, (n >> 1) & 1, w) && wait_bounded(s_full, n & 1, w);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* lse2 = stat + s * 256;
+      const float* dd = lse2 + 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {  // 32 query columns at a time
+        uint32_t sv[32], dp[32];
+        tmem_ld32(tbase + c * 32 + lane_off, sv);
+        tmem_ld32(tbase + 128 + c * 32 + lane_off, dp);
+        tmem_ld_wait(sv);
+        tmem_ld_wait(dp);
+        uint32_t pp[16], ps[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pr[2], ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qi = c * 32 + e + u;
+            const int q = qb + qi;
+            float x = __uint_as_float(sv[e + u]) * p.scale_log2;
+            if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
+            pr[u] = mg.allowed(q, k) ? ex2(x - lse2[qi]) : 0.f;
+            ds[u] = pr[u] * (__uint_as_float(dp[e + u]) - dd[qi]);
+          }
+          pp[e / 2] = pack2<BF16>(pr[0], pr[1]);
+          ps[e / 2] = pack2<BF16>(ds[0], ds[1]);
+        }
+        tmem_st16(tbase + c * 16 + lane_off, pp);        // P^T over read columns of S^T
+        tmem_st16(tbase + 128 + c * 16 + lane_off, ps);  // dS^T over read columns of dP^T
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    // ---- epilogue: dV, scale * dK -> 16-bit
+    if (ok && n_iter > 0) ok = wait_bounded(done, 0, w);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const bool row_ok = k < p.Sk;
+      const int64_t ro = ((static_cast<int64_t>(b) * p.Sk + k) * p.Hkv + hk) * D;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+        uint16_t* dst = static_cast<uint16_t*>(which ? p.dk : p.dv) + ro;
+        const float mul = which ? p.scale : 1.f;
+#pragma unroll 1
+        for (int c2 = 0; c2 < D / 32; ++c2) {
+          uint32_t o[32];
+          if (n_iter > 0) {
+            tmem_ld32(tbase + 256 + which * D + c2 * 32 + lane_off, o);
+            tmem_ld_wait(o);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * mul, __uint_as_float(o[2 * e + 1]) * mul);
+          if (row_ok) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c2 * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tbase, Cfg::kTmemCols);
+  }
+}
+
+// One CTA per (128-query block, head h, batch b).
+template <int D, bool BF16, bool ALIBI>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const BwdParams p) {
+  using Cfg = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int q0 = blockIdx.x * 128;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int hk = h / p.G;
+  const MaskGeo mg = mask_geo(p);
+  // keys seen by some query of [q0, q_last]
+  const int q_last = min(q0 + 127, p.Sq - 1);
+  const int k_begin = mg.has_left ? max(0, q0 + mg.off - mg.wl) : 0;
+  const int k_end = mg.has_right ? min(q_last + mg.off + mg.right, p.Sk - 1) + 1 : p.Sk;
+  const int j_lo = k_begin / 128;
+  const int n_blk = (q0 < p.Sq && k_end > k_begin) ? (k_end + 127) / 128 - j_lo : 0;
+
+  uint8_t* fixA = smem + Cfg::kFixA;  // Q_i
+  uint8_t* fixB = smem + Cfg::kFixB;  // dO_i
+  uint8_t* stage = smem + Cfg::kStage;  // slot s: K_j at s * 2 tiles, V_j after it
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
+  uint64_t* fix_full = bars;
+  uint64_t* full = bars + 1;
+  uint64_t* empty = bars + 3;
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* done = bars + 9;
+  uint64_t* drain = bars + 10;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
+
+  if (warp == 4 && lane == 0) {
+    mbar_init(fix_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_holder, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+  const WaitCtx w{abort_flag, p.status, p.timeout_ns};
+
+  if (warp == 4) {
+    // ======================================================== TMA producer
+    if (lane == 0 && n_blk > 0) {
+      tma_prefetch_map(&tmQ);
+      tma_prefetch_map(&tmK);
+      tma_prefetch_map(&tmV);
+      tma_prefetch_map(&tmDO);
+      mbar_arrive_expect_tx(fix_full, 2 * Cfg::kTileBytes);
+      for (int c = 0; c < Cfg::kChunks; ++c) {
+        tma_load_4d(fixA + c * Cfg::kChunkBytes, &tmQ, fix_full, c * 64, q0, h, b);
+        tma_load_4d(fixB + c * Cfg::kChunkBytes, &tmDO, fix_full, c * 64, q0, h, b);
+      }
+      int last[2] = {-1, -1};
+      for (int it = 0; it < n_blk; ++it) {
+        const int s = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        const int kb = (j_lo + it) * 128;
+        if (!wait_bounded(empty + s, ph ^ 1, w)) break;
+        mbar_arrive_expect_tx(full + s, 2 * Cfg::kTileBytes);
+        uint8_t* st = stage + s * 2 * Cfg::kTileBytes;
+        for (int c = 0; c < Cfg::kChunks; ++c) {
+          tma_load_4d(st + c * Cfg::kChunkBytes, &tmK, full + s, c * 64, kb, hk, b);
+          tma_load_4d(st + Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmV, full + s, c * 64, kb, hk,
+                      b);
+        }
+        last[s] = ph;
+      }
+      if (*abort_flag) {
+        wait_drain_bwd(fix_full, 0, p.timeout_ns);
+        for (int s = 0; s < 2; ++s)
+          if (last[s] >= 0) wait_drain_bwd(full + s, last[s], p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ======================================================== MMA issuer
+    if (lane == 0 && n_blk > 0) {
+      constexpr uint32_t idesc_s = f16_idesc(BF16, 128, 128, false, false);
+      constexpr uint32_t idesc_acc = f16_idesc(BF16, 128, D, false, true);
+      const uint64_t dQk = sw128_desc(smem_u32(fixA), 16, 1024);
+      const uint64_t dOk = sw128_desc(smem_u32(fixB), 16, 1024);
+      bool ok = wait_bounded(fix_full, 0, w);
+      for (int it = 0; it < n_blk && ok; ++it) {
+        const int s = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (!(ok = wait_bounded(full + s, ph, w))) break;
+        tc_fence_after();
+        const uint32_t sk = smem_u32(stage + s * 2 * Cfg::kTileBytes);
+        const uint32_t sv = sk + Cfg::kTileBytes;
+        fwd_issue_qk<D>(tbase, dQk, sw128_desc(sk, 16, 1024), idesc_s);         // S
+        fwd_issue_qk<D>(tbase + 128, dOk, sw128_desc(sv, 16, 1024), idesc_s);   // dP
+        tc_commit(s_full);
+        if (!(ok = wait_bounded(p_full, it & 1, w))) break;
+        tc_fence_after();
+        // dQ += dS K_j: B = K_j MN-major (rows are keys, the head dim contiguous)
+        fwd_issue_pv<D>(tbase + 256, tbase, sw128_desc(sk, Cfg::kChunkBytes, 1024), idesc_acc,
+                        it > 0);
+        tc_commit(empty + s);
+      }
+      if (ok) tc_commit(done);
+      tc_commit(drain);
+      wait_drain_bwd(drain, 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ======================================================== compute
+    const int r = threadIdx.x;  // query row within the block = TMEM lane
+    const int q = q0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int64_t idx = (static_cast<int64_t>(b) * p.H + h) * p.Sq + q;
+    const float lse2 = (q < p.Sq) ? p.lse[idx] * kBwdLog2e : INFINITY;
+    const float dd = (q < p.Sq) ? p.dvec[idx] : 0.f;
+    const float slope2 = ALIBI ? p.alibi[h] * kBwdLog2e : 0.f;
+    bool ok = true;
+    for (int it = 0; it < n_blk; ++it) {
+      const int kb = (j_lo + it) * 128;
+      ok = wait_bounded(s_full, it & 1, w);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {  // 32 key columns at a time
+        uint32_t sv[32], dp[32];
+        tmem_ld32(tbase + c * 32 + lane_off, sv);
+        tmem_ld32(tbase + 128 + c * 32 + lane_off, dp);
+        tmem_ld_wait(sv);
+        tmem_ld_wait(dp);
+        uint32_t ps[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int k = kb + c * 32 + e + u;
+            float x = __uint_as_float(sv[e + u]) * p.scale_log2;
+            if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
+            const float pr = mg.allowed(q, k) ? ex2(x - lse2) : 0.f;
+            ds[u] = pr * (__uint_as_float(dp[e + u]) - dd);
+          }
+          ps[e / 2] = pack2<BF16>(ds[0], ds[1]);
+        }
+        tmem_st16(tbase + c * 16 + lane_off, ps);  // dS over read columns of S
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    // ---- epilogue: scale * dQ -> 16-bit
+    if (ok && n_blk > 0) ok = wait_bounded(done, 0, w);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      uint16_t* dst = static_cast<uint16_t*>(p.dq) +
+                      ((static_cast<int64_t>(b) * p.Sq + q) * p.H + h) * D;
+#pragma unroll 1
+      for (int c2 = 0; c2 < D / 32; ++c2) {
+        uint32_t o[32];
+        if (n_blk > 0) {
+          tmem_ld32(tbase + 256 + c2 * 32 + lane_off, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * p.scale,
+                              __uint_as_float(o[2 * e + 1]) * p.scale);
+        if (q < p.Sq) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c2 * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tbase, Cfg::kTmemCols);
+  }
+}
+
+template <int D, bool BF16, bool ALIBI>
+cudaError_t launch_bwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+  using Cfg = BwdCfg<D>;
+  const int64_t rows = static_cast<int64_t>(p.B) * p.Sq * p.H;
+  bwd_dot_kernel<D, BF16><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  auto kkv = bwd_dkdv_kernel<D, BF16, ALIBI>;
+  auto kq = bwd_dq_kernel<D, BF16, ALIBI>;
+  if ((e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Cfg::kSmemAlloc)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Cfg::kSmemAlloc)) != cudaSuccess)
+    return e;
+  const dim3 gkv((p.Sk + 127) / 128, p.Hkv, p.B);
+  kkv<<<gkv, kBwdThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const dim3 gq((p.Sq + 127) / 128, p.H, p.B);
+  kq<<<gq, kBwdThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const BwdParams& p, bool bf16, int d,
+                       cudaStream_t stream) {
+  const bool al = p.alibi != nullptr;
+#define FA_BWD_CASE(DD, BF, AL) \
+  if (d == DD && bf16 == BF && al == AL) return launch_bwd_inst<DD, BF, AL>(tq, tk, tv, tdo, p, stream);
+  FA_BWD_CASE(64, false, false)
+  FA_BWD_CASE(64, false, true)
+  FA_BWD_CASE(64, true, false)
+  FA_BWD_CASE(64, true, true)
+  FA_BWD_CASE(128, false, false)
+  FA_BWD_CASE(128, false, true)
+  FA_BWD_CASE(128, true, false)
+  FA_BWD_CASE(128, true, true)
+#undef FA_BWD_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fa

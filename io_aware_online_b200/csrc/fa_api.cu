@@ -597,6 +597,98 @@ static int kvcache_impl(const void* q, const void* k_cache, const void* v_cache,
   return FA_OK;
 }
 
+size_t fa_bwd_workspace_size(int batch, int seqlen_q, int num_heads) {
+  if (batch <= 0 || seqlen_q <= 0 || num_heads <= 0) return 256;
+  const size_t need = static_cast<size_t>(batch) * num_heads * seqlen_q * sizeof(float);
+  return (need + 255) / 256 * 256;
+}
+
+int fa_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out,
+           const float* lse, void* dq, void* dk, void* dv, int dtype, int batch, int seqlen_q,
+           int seqlen_k, int num_heads, int num_heads_k, int head_dim, float softmax_scale,
+           int causal, int window_left, int window_right, float softcap,
+           const float* alibi_slopes, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  int rc = check_common(dtype, head_dim, num_heads, num_heads_k, window_left, window_right, softcap);
+  if (rc != FA_OK) return rc;
+  if (softcap > 0.f)
+    return fail(FA_ERR_UNSUPPORTED, "fa_bwd: softcap is not supported by the backward pass");
+  if (!dout || !q || !k || !v || !out || !lse || !dq || !dk || !dv)
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd: every tensor argument must be non-NULL");
+  if (!aligned16(dout) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd: 16-byte aligned tensors (lse 4-byte) required");
+  if (batch < 0 || seqlen_q < 0 || seqlen_k < 0)
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd: negative size");
+  float scale;
+  if ((rc = resolve_scale(softmax_scale, head_dim, &scale)) != FA_OK) return rc;
+  const int H = num_heads, Hkv = num_heads_k, d = head_dim;
+  const size_t need = fa_bwd_workspace_size(batch, seqlen_q, H);
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
+    return fail(FA_ERR_WORKSPACE, "fa_bwd: needs %zu bytes of 16-byte aligned workspace (got %zu)",
+                need, workspace_bytes);
+  if (batch == 0 || (seqlen_q == 0 && seqlen_k == 0)) return FA_OK;
+  if (seqlen_q == 0 || seqlen_k == 0) {  // nothing attends: every gradient is zero
+    cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+    cudaError_t e0 = cudaSuccess;
+    if (seqlen_k > 0) {
+      const size_t kv = static_cast<size_t>(batch) * seqlen_k * Hkv * d * 2;
+      if ((e0 = cudaMemsetAsync(dk, 0, kv, s0)) == cudaSuccess) e0 = cudaMemsetAsync(dv, 0, kv, s0);
+    } else {
+      e0 = cudaMemsetAsync(dq, 0, static_cast<size_t>(batch) * seqlen_q * H * d * 2, s0);
+    }
+    return e0 == cudaSuccess ? FA_OK : cuda_fail(e0, "fa_bwd zero fill");
+  }
+  if (batch > 65535 || H > 65535 || (seqlen_q + 127) / 128 > 65535 || (seqlen_k + 127) / 128 > 65535)
+    return fail(FA_ERR_UNSUPPORTED, "fa_bwd: sizes above the grid limits");
+  if ((rc = get_encoder()) != FA_OK) return rc;
+  unsigned int* status = nullptr;
+  if ((rc = device_state(nullptr, &status, nullptr)) != FA_OK) return rc;
+  CUtensorMap tq, tk, tv, tdo;
+  const uint32_t box[4] = {64, 128, 1, 1};
+  {
+    const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(seqlen_q),
+                              static_cast<uint64_t>(H), static_cast<uint64_t>(batch)};
+    const uint64_t st[3] = {static_cast<uint64_t>(H) * d * 2, static_cast<uint64_t>(d) * 2,
+                            static_cast<uint64_t>(seqlen_q) * H * d * 2};
+    if ((rc = encode_4d(&tq, q, dims, st, box, "q")) != FA_OK) return rc;
+    if ((rc = encode_4d(&tdo, dout, dims, st, box, "dout")) != FA_OK) return rc;
+  }
+  {
+    const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(seqlen_k),
+                              static_cast<uint64_t>(Hkv), static_cast<uint64_t>(batch)};
+    const uint64_t st[3] = {static_cast<uint64_t>(Hkv) * d * 2, static_cast<uint64_t>(d) * 2,
+                            static_cast<uint64_t>(seqlen_k) * Hkv * d * 2};
+    if ((rc = encode_4d(&tk, k, dims, st, box, "k")) != FA_OK) return rc;
+    if ((rc = encode_4d(&tv, v, dims, st, box, "v")) != FA_OK) return rc;
+  }
+  fa::BwdParams p{};
+  p.out = out;
+  p.dout = dout;
+  p.lse = lse;
+  p.dvec = static_cast<float*>(workspace);
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.B = batch;
+  p.Sq = seqlen_q;
+  p.Sk = seqlen_k;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.alibi = alibi_slopes;
+  p.causal = causal ? 1 : 0;
+  p.wl = window_left;
+  p.wr = window_right;
+  p.status = status;
+  p.timeout_ns = timeout_ns();
+  const cudaError_t e = fa::launch_bwd(tq, tk, tv, tdo, p, dtype == FA_BF16, d,
+                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e, "fa_bwd launch");
+}
+
 int fa_selftest_wait_timeout(int timeout_ms, void* stream) {
   g_err.clear();
   if (timeout_ms <= 0 || timeout_ms > 10000)

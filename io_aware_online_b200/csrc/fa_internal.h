@@ -92,6 +92,28 @@ struct CombineParams {
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
+// ---------------------------------------------------------------- backward
+struct BwdParams {
+  const void* out;                 // forward output O [B, Sq, H, D] (16-bit, contiguous)
+  const void* dout;                // dO, same layout
+  const float* lse;                // [B, H, Sq] natural-log LSE of the forward
+  float* dvec;                     // [B, H, Sq] D = rowsum(dO * O) (workspace)
+  void* dq;                        // [B, Sq, H, D] 16-bit
+  void* dk;                        // [B, Sk, Hkv, D] 16-bit
+  void* dv;
+  int B, Sq, Sk, H, Hkv, G;
+  float scale;                     // softmax_scale
+  float scale_log2;                // softmax_scale * log2(e)
+  const float* alibi;              // [H] or NULL
+  int causal, wl, wr;
+  unsigned int* status;
+  uint64_t timeout_ns;
+};
+
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const BwdParams& p, bool bf16, int d,
+                       cudaStream_t stream);
+
 cudaError_t launch_wait_timeout_selftest(unsigned int* status, uint64_t timeout_ns,
                                          cudaStream_t stream);
 

@@ -47,9 +47,10 @@ def _allowed(Sq, Sk, causal, window):
 
 
 def attention_backward(q, k, v, do, *, scale=None, causal=False, window=(-1, -1),
-                       alibi_slopes=None):
+                       alibi_slopes=None, return_probs=False):
     """q [B, Sq, H, d], k/v [B, Sk, Hkv, d], do like q.
-    Returns (dq like q, dk, dv like k, o like q, lse [B, H, Sq]) in float64."""
+    Returns (dq like q, dk, dv like k, o like q, lse [B, H, Sq]) in float64, and
+    with return_probs also P and dS [B, H, Sq, Sk]."""
     q, k, v, do = _np64(q), _np64(k), _np64(v), _np64(do)
     B, Sq, H, d = q.shape
     Sk, Hkv = k.shape[1], k.shape[2]
@@ -64,6 +65,8 @@ def attention_backward(q, k, v, do, *, scale=None, causal=False, window=(-1, -1)
     dv = np.zeros_like(v)
     o = np.zeros_like(q)
     lse = np.full((B, H, Sq), -np.inf)
+    probs = np.zeros((B, H, Sq, Sk)) if return_probs else None
+    dss = np.zeros((B, H, Sq, Sk)) if return_probs else None
     for b in range(B):
         for h in range(H):
             hk = h // G
@@ -85,6 +88,11 @@ def attention_backward(q, k, v, do, *, scale=None, causal=False, window=(-1, -1)
             dk[b, :, hk] += scale * (dS.T @ Q)
             dv[b, :, hk] += P.T @ dO
             o[b, :, h] = O
+            if return_probs:
+                probs[b, h] = P
+                dss[b, h] = dS
             lse[b, h] = np.where(live, m[:, 0] + np.log(np.where(live, den[:, 0], 1.0)),
                                  -np.inf)
+    if return_probs:
+        return dq, dk, dv, o, lse, probs, dss
     return dq, dk, dv, o, lse
