@@ -330,6 +330,72 @@ APPEND = dict(B=4, S_new=8192, Hkv=8, d=128, dtype="bf16", page=256)
 FP8 = dict(B=4, S=8192, H=32, Hkv=32, d=128, dtype="e4m3", causal=True)
 
 
+# backward (fa_bwd): the d=128 causal prefill point
+BWD = dict(B=4, S=4096, H=32, Hkv=32, d=128, dtype="bf16", causal=True)
+
+
+def run_bwd(args, rank, world, local):
+    """--only bwd: time fa_bwd (D pre-pass + dK/dV + dQ kernels).  Algorithmic work:
+    the five products of the backward (S, dP, dV, dK, dQ), 10 d FLOPs per allowed
+    (query, key) pair, i.e. 2.5x the forward's."""
+    import io_aware_online_b200 as fa
+    from io_aware_online_b200 import build as fa_build
+    fa_build.build()
+    fa.load()
+    dev = torch.device("cuda", local)
+    hbm_peak, tflops_peak, peak_src = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    c = BWD
+    dt = synth.DTYPES[c["dtype"]]
+    gen = torch.Generator(device=dev).manual_seed(3200 + rank)
+    shp_q = (c["B"], c["S"], c["H"], c["d"])
+    shp_k = (c["B"], c["S"], c["Hkv"], c["d"])
+    q = torch.randn(shp_q, generator=gen, device=dev).to(dt)
+    k = torch.randn(shp_k, generator=gen, device=dev).to(dt)
+    v = torch.randn(shp_k, generator=gen, device=dev).to(dt)
+    do = torch.randn(shp_q, generator=gen, device=dev).to(dt)
+    out, lse = fa.fa_fwd(q, k, v, causal=True, stream=stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.load().fa_bwd_workspace_size(c["B"], c["S"], c["H"]), dtype=torch.uint8,
+                     device=dev)
+    work = 10.0 * c["d"] * c["B"] * c["H"] * causal_pairs(c["S"], c["S"])
+
+    def call():
+        fa.fa_bwd(do, q, k, v, out, lse, causal=True, dq=dq, dk=dk, dv=dv, workspace=ws,
+                  stream=stream)
+    for _ in range(args.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with Clocks(dev.index if dev.index is not None else 0) as clk:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world)
+    achieved = work / (ms * 1e-3) / 1e12
+    return {"metric": "attn bwd TFLOPS (causal, dQ dK dV)", "value": round(achieved * world, 2),
+            "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": c["dtype"], "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": "bwd", **c, "l2": "flushed between steps (256 MiB write, "
+                       "untimed)", "parallelism": f"dp{world} (independent replicas)"},
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": tflops_peak,
+                         "unit": "TFLOP/s", "frac": round(achieved / tflops_peak, 4),
+                         "traffic": None,
+                         "kernel": "bwd_dot_kernel + bwd_dkdv_kernel + bwd_dq_kernel <128, bf16>",
+                         "peak_source": peak_src},
+            "gpu_launches": 3 * K, "clocks": clk.summary()}
+
+
 def run_fp8(args, rank, world, local):
     """--only fp8: time fa_fwd_fp8 on the d=128 causal prefill workload."""
     import io_aware_online_b200 as fa
@@ -558,7 +624,8 @@ def main():
     ap.add_argument("--num-splits", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "chunked", "append", "fp8"],
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "chunked", "append", "fp8",
+                                       "bwd"],
                     default="all",
                     help="time one part of the step (profiling / sweeps), or one of the "
                          "cache-update rows on its own workload (chunked, append)")
@@ -577,8 +644,9 @@ def main():
             if rank == 0:
                 print(json.dumps(run_reference(args, rank, world)), flush=True)
             return
-        if args.only in ("chunked", "append", "fp8"):
-            res = (run_fp8 if args.only == "fp8" else run_cache_rows)(args, rank, world, local)
+        if args.only in ("chunked", "append", "fp8", "bwd"):
+            fn = {"fp8": run_fp8, "bwd": run_bwd}.get(args.only, run_cache_rows)
+            res = fn(args, rank, world, local)
             if rank == 0:
                 print(json.dumps(res), flush=True)
             return

@@ -49,8 +49,8 @@ struct BwdCfg {
   static constexpr int kStage = 2 * kTileBytes;       // 2 stages x {A, B} streamed tiles
   static constexpr int kStat = kStage + 4 * kTileBytes;  // [2 slots][2][128] fp32
   static constexpr int kBarOff = kStat + 2 * 2 * 128 * 4;
-  // fix_full, full[2], empty[2], s_full, p_full, stat[2], done, drain
-  static constexpr int kNumBars = 11;
+  // fix_full, full[2], empty[2], s_full, p_full, stat[2], done, drain, dp_full, ds_full
+  static constexpr int kNumBars = 13;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   // room to align the base to 1 KiB; at least 116 KiB, so that one CTA fills an SM
@@ -70,6 +70,13 @@ struct MaskGeo {
     const int c = i + off;
     if (has_right && j > c + right) return false;
     if (has_left && j < c - wl) return false;
+    return true;
+  }
+  // every (query, key) of the 128 x 128 tile at (i0, j0) allowed: no mask needed
+  __device__ __forceinline__ bool tile_open(int i0, int j0) const {
+    if (i0 + 127 >= Sq || j0 + 127 >= Sk) return false;
+    if (has_right && j0 + 127 > i0 + off + right) return false;
+    if (has_left && j0 < i0 + 127 + off - wl) return false;
     return true;
   }
 };
@@ -133,9 +140,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int k0 = blockIdx.x * 128;
-  const int hk = blockIdx.y;
-  const int b = blockIdx.z;
+  // grid: KV heads fastest, key blocks slowest: under a causal mask key block 0
+  // is seen by every query block, so the heaviest CTAs start first
+  const int k0 = blockIdx.z * 128;
+  const int hk = blockIdx.x;
+  const int b = blockIdx.y;
   const MaskGeo mg = mask_geo(p);
   // query rows that see some key of [k0, k1)
   const int k1 = min(k0 + 128, p.Sk);
@@ -158,6 +167,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* statb = bars + 7;
   uint64_t* done = bars + 9;
   uint64_t* drain = bars + 10;
+  uint64_t* dp_full = bars + 11;
+  uint64_t* ds_full = bars + 12;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -169,7 +180,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(statb + s, 4);
     }
     mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
     mbar_init(p_full, 4);
+    mbar_init(ds_full, 4);
     mbar_init(done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -227,25 +240,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       constexpr uint32_t idesc_acc = f16_idesc(BF16, 128, D, false, true);
       const uint64_t dKk = sw128_desc(smem_u32(fixA), 16, 1024);  // K-major operands
       const uint64_t dVk = sw128_desc(smem_u32(fixB), 16, 1024);
-      bool ok = wait_bounded(fix_full, 0, w);
+      // Software pipeline, in issue order:
+      //   S^T(0), dP^T(0); per block n:
+      //   [P^T(n) ready] dV(n), S^T(n+1); [dS^T(n) ready] dK(n), dP^T(n+1)
+      // so the compute warps' dS^T(n) overlaps dV(n) and S^T(n+1), and their
+      // P^T(n+1) overlaps dK(n) and dP^T(n+1).  A product that overwrites a region
+      // (S^T(n+1) over P^T(n), dP^T(n+1) over dS^T(n)) is issued after the one
+      // reading it, and each commit covers every earlier product of this thread.
+      auto st_q = [&](int s) { return smem_u32(stage + s * 2 * Cfg::kTileBytes); };
+      bool ok = wait_bounded(fix_full, 0, w) && wait_bounded(full, 0, w);
+      if (ok) {
+        tc_fence_after();
+        fwd_issue_qk<D>(tbase, dKk, sw128_desc(st_q(0), 16, 1024), idesc_s);         // S^T(0)
+        tc_commit(s_full);
+        fwd_issue_qk<D>(tbase + 128, dVk, sw128_desc(st_q(0) + Cfg::kTileBytes, 16, 1024),
+                        idesc_s);                                                      // dP^T(0)
+        tc_commit(dp_full);
+      }
       for (int n = 0; n < n_iter && ok; ++n) {
         const int s = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
-        if (!(ok = wait_bounded(full + s, ph, w))) break;
-        tc_fence_after();
-        const uint32_t sq = smem_u32(stage + s * 2 * Cfg::kTileBytes);
+        const bool more = n + 1 < n_iter;
+        const uint32_t sq = st_q(s);
         const uint32_t sdo = sq + Cfg::kTileBytes;
-        fwd_issue_qk<D>(tbase, dKk, sw128_desc(sq, 16, 1024), idesc_s);          // S^T
-        fwd_issue_qk<D>(tbase + 128, dVk, sw128_desc(sdo, 16, 1024), idesc_s);   // dP^T
-        tc_commit(s_full);
         if (!(ok = wait_bounded(p_full, n & 1, w))) break;
         tc_fence_after();
         // B operands MN-major: rows are queries, the head dim contiguous
         fwd_issue_pv<D>(tbase + 256, tbase, sw128_desc(sdo, Cfg::kChunkBytes, 1024), idesc_acc,
-                        n > 0);                                                   // dV
+                        n > 0);                                                   // dV(n)
+        if (more) {
+          if (!(ok = wait_bounded(full + (s ^ 1), ((n + 1) >> 1) & 1, w))) break;
+          tc_fence_after();
+          fwd_issue_qk<D>(tbase, dKk, sw128_desc(st_q(s ^ 1), 16, 1024), idesc_s);  // S^T(n+1)
+          tc_commit(s_full);
+        }
+        if (!(ok = wait_bounded(ds_full, n & 1, w))) break;
+        tc_fence_after();
         fwd_issue_pv<D>(tbase + 256 + D, tbase + 128, sw128_desc(sq, Cfg::kChunkBytes, 1024),
-                        idesc_acc, n > 0);                                        // dK
+                        idesc_acc, n > 0);                                        // dK(n)
         tc_commit(empty + s);
+        if (more) {
+          fwd_issue_qk<D>(tbase + 128, dVk,
+                          sw128_desc(st_q(s ^ 1) + Cfg::kTileBytes, 16, 1024), idesc_s);  // dP^T(n+1)
+          tc_commit(dp_full);
+        }
       }
       if (ok) tc_commit(done);
       tc_commit(drain);
@@ -281,36 +318,65 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const float* lse2 = stat + s * 256;
       const float* dd = lse2 + 128;
-#pragma unroll 1
+      // phase 1: P^T (kept in fp32 registers), 16-bit copy over read columns of S^T
+      const bool open = mg.tile_open(qb, k0);  // uniform: the whole tile is unmasked
+      const float4* lse4 = reinterpret_cast<const float4*>(lse2);
+      float pf[128];
+#pragma unroll
       for (int c = 0; c < 4; ++c) {  // 32 query columns at a time
-        uint32_t sv[32], dp[32];
+        uint32_t sv[32];
         tmem_ld32(tbase + c * 32 + lane_off, sv);
-        tmem_ld32(tbase + 128 + c * 32 + lane_off, dp);
         tmem_ld_wait(sv);
-        tmem_ld_wait(dp);
-        uint32_t pp[16], ps[16];
+        uint32_t pp[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pr[2], ds[2];
+        for (int e = 0; e < 32; e += 4) {
+          const float4 l4 = lse4[(c * 32 + e) / 4];  // one broadcast load, four columns
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
+          for (int u = 0; u < 4; ++u) {
             const int qi = c * 32 + e + u;
             const int q = qb + qi;
             float x = __uint_as_float(sv[e + u]) * p.scale_log2;
             if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
-            pr[u] = mg.allowed(q, k) ? ex2(x - lse2[qi]) : 0.f;
-            ds[u] = pr[u] * (__uint_as_float(dp[e + u]) - dd[qi]);
+            pf[qi] = (open || mg.allowed(q, k)) ? ex2(x - lv[u]) : 0.f;
           }
-          pp[e / 2] = pack2<BF16>(pr[0], pr[1]);
-          ps[e / 2] = pack2<BF16>(ds[0], ds[1]);
+          pp[e / 2] = pack2<BF16>(pf[c * 32 + e], pf[c * 32 + e + 1]);
+          pp[e / 2 + 1] = pack2<BF16>(pf[c * 32 + e + 2], pf[c * 32 + e + 3]);
         }
-        tmem_st16(tbase + c * 16 + lane_off, pp);        // P^T over read columns of S^T
-        tmem_st16(tbase + 128 + c * 16 + lane_off, ps);  // dS^T over read columns of dP^T
+        tmem_st16(tbase + c * 16 + lane_off, pp);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
+      // phase 2: dS^T = P^T * (dP^T - D) over read columns of dP^T
+      ok = wait_bounded(dp_full, n & 1, w);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t dp[32];
+        tmem_ld32(tbase + 128 + c * 32 + lane_off, dp);
+        tmem_ld_wait(dp);
+        uint32_t ps[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const int qi = c * 32 + e;
+          const float4 d4 = reinterpret_cast<const float4*>(dd)[qi / 4];
+          ps[e / 2] = pack2<BF16>(pf[qi] * (__uint_as_float(dp[e]) - d4.x),
+                                  pf[qi + 1] * (__uint_as_float(dp[e + 1]) - d4.y));
+          ps[e / 2 + 1] = pack2<BF16>(pf[qi + 2] * (__uint_as_float(dp[e + 2]) - d4.z),
+                                      pf[qi + 3] * (__uint_as_float(dp[e + 3]) - d4.w));
+        }
+        tmem_st16(tbase + 128 + c * 16 + lane_off, ps);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full);
     }
     // ---- epilogue: dV, scale * dK -> 16-bit
     if (ok && n_iter > 0) ok = wait_bounded(done, 0, w);
@@ -367,9 +433,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int q0 = blockIdx.x * 128;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
+  // grid: heads fastest, query blocks slowest and last first (the last query
+  // block sees the most keys under a causal mask: heaviest CTAs start first)
+  const int q0 = (static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z)) * 128;
+  const int h = blockIdx.x;
+  const int b = blockIdx.y;
   const int hk = h / p.G;
   const MaskGeo mg = mask_geo(p);
   // keys seen by some query of [q0, q_last]
@@ -498,6 +566,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         break;
       }
       tc_fence_after();
+      const bool open = mg.tile_open(q0, kb);  // uniform: the whole tile is unmasked
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {  // 32 key columns at a time
         uint32_t sv[32], dp[32];
@@ -514,7 +583,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int k = kb + c * 32 + e + u;
             float x = __uint_as_float(sv[e + u]) * p.scale_log2;
             if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
-            const float pr = mg.allowed(q, k) ? ex2(x - lse2) : 0.f;
+            const float pr = (open || mg.allowed(q, k)) ? ex2(x - lse2) : 0.f;
             ds[u] = pr * (__uint_as_float(dp[e + u]) - dd);
           }
           ps[e / 2] = pack2<BF16>(ds[0], ds[1]);
@@ -581,10 +650,10 @@ cudaError_t launch_bwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const 
   if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 Cfg::kSmemAlloc)) != cudaSuccess)
     return e;
-  const dim3 gkv((p.Sk + 127) / 128, p.Hkv, p.B);
+  const dim3 gkv(p.Hkv, p.B, (p.Sk + 127) / 128);
   kkv<<<gkv, kBwdThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const dim3 gq((p.Sq + 127) / 128, p.H, p.B);
+  const dim3 gq(p.H, p.B, (p.Sq + 127) / 128);
   kq<<<gq, kBwdThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError();
 }
