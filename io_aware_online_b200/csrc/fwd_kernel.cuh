@@ -145,8 +145,10 @@ __device__ __forceinline__ void fwd_issue_pv(uint32_t d_tmem, uint32_t a_tmem, u
 }
 
 // FP8: E4M3 Q, K, V (both products on kind::f8f6f4, P rounded to E4M3), bf16 output
-// (BF16 must then be true).
-template <int D, int T, bool BF16, bool SOFTCAP, bool ALIBI, int EMU, bool FP8 = false>
+// (BF16 must then be true).  KV: K/V from a KV cache (FwdParams::kv_mode); a
+// compile-time switch, so the dense kernels carry none of its code.
+template <int D, int T, bool BF16, bool SOFTCAP, bool ALIBI, int EMU, bool FP8 = false,
+          bool KV = false>
 __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
                                   FwdCfg<D, T, FP8 ? 1 : 2>::kMinBlocks)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -176,7 +178,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
     Sq_b = p.cu_q[b + 1] - q0;
     k0 = p.cu_k[b];
     Sk_b = p.cu_k[b + 1] - k0;
-  } else if (p.kv_mode) {
+  } else if (KV) {
     Sk_b = ((p.cache_seqlens != nullptr) ? p.cache_seqlens[b] : p.Sk) + p.k_add;
     // a length the cache cannot hold would read past the block table: clamp, report
     const int cap = (p.block_table != nullptr) ? p.max_blocks * p.page_size : p.Sk;
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
         const int s = it % ST;
         const uint32_t ph = (it / ST) & 1;
         const int j = j_lo + it;
-        if (!p.kv_mode) {
+        if constexpr (!KV) {
           if (!wait_bounded(k_empty + s, ph ^ 1, w)) break;
           mbar_arrive_expect_tx(k_full + s, Cfg::kTileBytes);
           for (int c = 0; c < Cfg::kChunks; ++c)
@@ -654,7 +656,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
       // the page tail (or an unloaded half) holds; P is 0 there, but 0 * NaN is
       // NaN in P.V, so this warp zeroes its 32 rows of them before releasing P
       // (both tiles' warps write the same zeros)
-      if (p.kv_mode && kb + kBN > Sk_b) {
+      if (KV && kb + kBN > Sk_b) {
         const int s = it % ST;
         ok = wait_bounded(v_full + s, (it / ST) & 1, w);
         if (!__all_sync(0xffffffffu, ok)) {

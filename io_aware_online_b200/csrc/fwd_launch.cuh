@@ -8,11 +8,12 @@
 
 namespace fa {
 
-template <int D, int T, bool BF16, bool SOFTCAP, bool ALIBI, int EMU, bool FP8 = false>
+template <int D, int T, bool BF16, bool SOFTCAP, bool ALIBI, int EMU, bool FP8 = false,
+          bool KV = false>
 cudaError_t launch_fwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int batch, int rows_q, cudaStream_t stream) {
   using Cfg = FwdCfg<D, T, FP8 ? 1 : 2>;
-  auto kern = fwd_kernel<D, T, BF16, SOFTCAP, ALIBI, EMU, FP8>;
+  auto kern = fwd_kernel<D, T, BF16, SOFTCAP, ALIBI, EMU, FP8, KV>;
   constexpr int smem = Cfg::kSmemAlloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess && T == 1)  // room for two CTAs per SM
@@ -56,6 +57,22 @@ cudaError_t launch_fwd_dtype(const CUtensorMap& tq, const CUtensorMap& tk, const
                              cudaStream_t stream) {
   const bool sc = p.softcap_log2 > 0.f;
   const bool al = p.alibi != nullptr;
+  if (p.kv_mode) {  // KV-cache mode: two tiles, the default exponential split
+#define FA_FWD_KV_CASE(DD, SC, AL, EM)                                                     \
+  if (d == DD && sc == SC && al == AL)                                                     \
+    return launch_fwd_inst<DD, 2, BF16, SC, AL, EM, false, true>(tq, tk, tv, p, batch, rows_q, \
+                                                                 stream);
+    FA_FWD_KV_CASE(64, false, false, 2)
+    FA_FWD_KV_CASE(64, true, false, 0)
+    FA_FWD_KV_CASE(64, false, true, 0)
+    FA_FWD_KV_CASE(64, true, true, 0)
+    FA_FWD_KV_CASE(128, false, false, 0)
+    FA_FWD_KV_CASE(128, true, false, 0)
+    FA_FWD_KV_CASE(128, false, true, 0)
+    FA_FWD_KV_CASE(128, true, true, 0)
+#undef FA_FWD_KV_CASE
+    return cudaErrorInvalidValue;
+  }
   const int emu = (sc || al) ? 0 : exp2_emu_choice(d);
   const int tiles = (d == 64) ? fwd_tiles_choice() : 2;
 #define FA_FWD_CASE(DD, TT, SC, AL, EM)                                                    \
