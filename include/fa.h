@@ -247,8 +247,9 @@ FA_API int fa_fwd_kvcache_append(const void *q, void *k_cache, void *v_cache, co
                                  void *stream);
 
 /*
- * fa_bwd_workspace_size -- bytes of device scratch fa_bwd needs: batch *
- * num_heads * seqlen_q fp32 values (D = rowsum(dO * O)), rounded up to 256.
+ * fa_bwd_workspace_size -- bytes of device scratch fa_bwd needs: two fp32 arrays
+ * (D = rowsum(dO * O) and LSE * log2 e) of batch * num_heads rows of seqlen_q
+ * rounded up to 4 values, the total rounded up to 256 bytes.
  */
 FA_API size_t fa_bwd_workspace_size(int batch, int seqlen_q, int num_heads);
 

@@ -124,7 +124,9 @@ __global__ void __launch_bounds__(256) bwd_dot_kernel(const BwdParams p) {
     const int64_t bi = row / p.H;  // b * Sq + i
     const int i = static_cast<int>(bi % p.Sq);
     const int b = static_cast<int>(bi / p.Sq);
-    p.dvec[(static_cast<int64_t>(b) * p.H + h) * p.Sq + i] = acc;
+    const int64_t bh = static_cast<int64_t>(b) * p.H + h;
+    p.dvec[bh * p.sq_pad + i] = acc;
+    p.lse2[bh * p.sq_pad + i] = p.lse[bh * p.Sq + i] * kBwdLog2e;  // base-2 LSE for P
   }
 }
 
@@ -133,6 +135,7 @@ template <int D, bool BF16, bool ALIBI>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmD,
                     const BwdParams p) {
   using Cfg = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -164,7 +167,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* empty = bars + 3;
   uint64_t* s_full = bars + 5;
   uint64_t* p_full = bars + 6;
-  uint64_t* statb = bars + 7;
   uint64_t* done = bars + 9;
   uint64_t* drain = bars + 10;
   uint64_t* dp_full = bars + 11;
@@ -177,7 +179,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
-      mbar_init(statb + s, 4);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
@@ -217,13 +218,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int h = hk * p.G + n / nqb;
         const int qb = (i_lo + n % nqb) * 128;
         if (!wait_bounded(empty + s, ph ^ 1, w)) break;
-        mbar_arrive_expect_tx(full + s, 2 * Cfg::kTileBytes);
+        // Q_i, dO_i and the block's column statistics (LSE * log2 e and D; zero past
+        // the end of the rows, where the mask keeps P at 0)
+        mbar_arrive_expect_tx(full + s, 2 * Cfg::kTileBytes + 2 * 128 * 4);
         uint8_t* st = stage + s * 2 * Cfg::kTileBytes;
         for (int c = 0; c < Cfg::kChunks; ++c) {
           tma_load_4d(st + c * Cfg::kChunkBytes, &tmQ, full + s, c * 64, qb, h, b);
           tma_load_4d(st + Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmDO, full + s, c * 64, qb, h,
                       b);
         }
+        tma_load_2d(stat + s * 256, &tmL, full + s, qb, b * p.H + h);
+        tma_load_2d(stat + s * 256 + 128, &tmD, full + s, qb, b * p.H + h);
         last[s] = ph;
       }
       if (*abort_flag) {  // let this CTA's own copies land before the smem goes away
@@ -300,17 +305,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int h = hk * p.G + n / nqb;
       const int qb = (i_lo + n % nqb) * 128;
       const float slope2 = ALIBI ? p.alibi[h] * kBwdLog2e : 0.f;
-      // column statistics of this query block: thread r provides query qb + r
-      {
-        const int q = qb + r;
-        const int64_t idx = (static_cast<int64_t>(b) * p.H + h) * p.Sq + q;
-        float* slot = stat + s * 256;
-        slot[r] = (q < p.Sq) ? p.lse[idx] * kBwdLog2e : INFINITY;  // P = 0 past the end
-        slot[128 + r] = (q < p.Sq) ? p.dvec[idx] : 0.f;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(statb + s);
-      }
-      ok = wait_bounded(statb + s, (n >> 1) & 1, w) && wait_bounded(s_full, n & 1, w);
+      // the stage (with this block's column statistics) has landed, and S^T is ready
+      ok = wait_bounded(full + s, (n >> 1) & 1, w) && wait_bounded(s_full, n & 1, w);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -553,8 +549,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int r = threadIdx.x;  // query row within the block = TMEM lane
     const int q = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const int64_t idx = (static_cast<int64_t>(b) * p.H + h) * p.Sq + q;
-    const float lse2 = (q < p.Sq) ? p.lse[idx] * kBwdLog2e : INFINITY;
+    const int64_t idx = (static_cast<int64_t>(b) * p.H + h) * p.sq_pad + q;
+    const float lse2 = (q < p.Sq) ? p.lse2[idx] : INFINITY;
     const float dd = (q < p.Sq) ? p.dvec[idx] : 0.f;
     const float slope2 = ALIBI ? p.alibi[h] * kBwdLog2e : 0.f;
     bool ok = true;
@@ -636,7 +632,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 template <int D, bool BF16, bool ALIBI>
 cudaError_t launch_bwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+                            const CUtensorMap& tdo, const CUtensorMap& tl, const CUtensorMap& td,
+                            const BwdParams& p, cudaStream_t stream) {
   using Cfg = BwdCfg<D>;
   const int64_t rows = static_cast<int64_t>(p.B) * p.Sq * p.H;
   bwd_dot_kernel<D, BF16><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
@@ -651,7 +648,7 @@ cudaError_t launch_bwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const 
                                 Cfg::kSmemAlloc)) != cudaSuccess)
     return e;
   const dim3 gkv(p.Hkv, p.B, (p.Sk + 127) / 128);
-  kkv<<<gkv, kBwdThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
+  kkv<<<gkv, kBwdThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, tl, td, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const dim3 gq(p.H, p.B, (p.Sq + 127) / 128);
   kq<<<gq, kBwdThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
@@ -661,11 +658,12 @@ cudaError_t launch_bwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const 
 }  // namespace
 
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdParams& p, bool bf16, int d,
-                       cudaStream_t stream) {
+                       const CUtensorMap& tdo, const CUtensorMap& tl, const CUtensorMap& td,
+                       const BwdParams& p, bool bf16, int d, cudaStream_t stream) {
   const bool al = p.alibi != nullptr;
 #define FA_BWD_CASE(DD, BF, AL) \
-  if (d == DD && bf16 == BF && al == AL) return launch_bwd_inst<DD, BF, AL>(tq, tk, tv, tdo, p, stream);
+  if (d == DD && bf16 == BF && al == AL)                                                   \
+    return launch_bwd_inst<DD, BF, AL>(tq, tk, tv, tdo, tl, td, p, stream);
   FA_BWD_CASE(64, false, false)
   FA_BWD_CASE(64, false, true)
   FA_BWD_CASE(64, true, false)

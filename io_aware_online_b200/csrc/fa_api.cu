@@ -597,10 +597,27 @@ static int kvcache_impl(const void* q, const void* k_cache, const void* v_cache,
   return FA_OK;
 }
 
+// Backward workspace: D and LSE * log2(e), each [batch * num_heads rows, seqlen_q
+// rounded up to 4] fp32 (16-byte rows for the tensor maps that load them).
 size_t fa_bwd_workspace_size(int batch, int seqlen_q, int num_heads) {
   if (batch <= 0 || seqlen_q <= 0 || num_heads <= 0) return 256;
-  const size_t need = static_cast<size_t>(batch) * num_heads * seqlen_q * sizeof(float);
-  return (need + 255) / 256 * 256;
+  const size_t half = static_cast<size_t>(batch) * num_heads * ((seqlen_q + 3) / 4 * 4) *
+                      sizeof(float);
+  return (2 * half + 255) / 256 * 256;
+}
+
+// 2-D fp32 tensor map over [rows, cols] with a row stride in bytes, box {128, 1}.
+static int encode_vec_rows(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t rows,
+                           uint64_t stride_bytes, const char* what) {
+  cuuint64_t gd[2] = {cols, rows};
+  cuuint64_t gs[1] = {stride_bytes};
+  cuuint32_t bx[2] = {128, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), gd, gs,
+                        bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_INVALID_ARG, "%s: tensor map encoding failed (%d)", what, (int)r);
+  return FA_OK;
 }
 
 int fa_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out,
@@ -662,11 +679,23 @@ int fa_bwd(const void* dout, const void* q, const void* k, const void* v, const 
     if ((rc = encode_4d(&tk, k, dims, st, box, "k")) != FA_OK) return rc;
     if ((rc = encode_4d(&tv, v, dims, st, box, "v")) != FA_OK) return rc;
   }
+  const int sq_pad = (seqlen_q + 3) / 4 * 4;
+  float* dvec = static_cast<float*>(workspace);
+  float* lse2 = dvec + static_cast<size_t>(batch) * H * sq_pad;
+  CUtensorMap tl, td;  // rows: the true length, so columns past the end load as 0
+  if ((rc = encode_vec_rows(&tl, lse2, seqlen_q, static_cast<uint64_t>(batch) * H,
+                            static_cast<uint64_t>(sq_pad) * 4, "lse workspace")) != FA_OK)
+    return rc;
+  if ((rc = encode_vec_rows(&td, dvec, seqlen_q, static_cast<uint64_t>(batch) * H,
+                            static_cast<uint64_t>(sq_pad) * 4, "D workspace")) != FA_OK)
+    return rc;
   fa::BwdParams p{};
   p.out = out;
   p.dout = dout;
   p.lse = lse;
-  p.dvec = static_cast<float*>(workspace);
+  p.dvec = dvec;
+  p.lse2 = lse2;
+  p.sq_pad = sq_pad;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
@@ -684,7 +713,7 @@ int fa_bwd(const void* dout, const void* q, const void* k, const void* v, const 
   p.wr = window_right;
   p.status = status;
   p.timeout_ns = timeout_ns();
-  const cudaError_t e = fa::launch_bwd(tq, tk, tv, tdo, p, dtype == FA_BF16, d,
+  const cudaError_t e = fa::launch_bwd(tq, tk, tv, tdo, tl, td, p, dtype == FA_BF16, d,
                                        static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : cuda_fail(e, "fa_bwd launch");
 }

@@ -98,6 +98,8 @@ struct BwdParams {
   const void* dout;                // dO, same layout
   const float* lse;                // [B, H, Sq] natural-log LSE of the forward
   float* dvec;                     // [B, H, Sq] D = rowsum(dO * O) (workspace)
+  float* lse2;                     // [B, H, Sq] LSE * log2(e) (workspace, after dvec)
+  int sq_pad;                      // row stride of dvec / lse2: Sq rounded up to 4
   void* dq;                        // [B, Sq, H, D] 16-bit
   void* dk;                        // [B, Sk, Hkv, D] 16-bit
   void* dv;
@@ -111,8 +113,8 @@ struct BwdParams {
 };
 
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdParams& p, bool bf16, int d,
-                       cudaStream_t stream);
+                       const CUtensorMap& tdo, const CUtensorMap& tl, const CUtensorMap& td,
+                       const BwdParams& p, bool bf16, int d, cudaStream_t stream);
 
 cudaError_t launch_wait_timeout_selftest(unsigned int* status, uint64_t timeout_ns,
                                          cudaStream_t stream);
