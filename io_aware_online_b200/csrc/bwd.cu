@@ -18,10 +18,10 @@
 //                    shared memory while the key blocks stream past; per block
 //                      S = Q_i K_j^T, dP = dO_i V_j^T, dS -> 16-bit,
 //                      dQ += dS K_j                           (tcgen05)
-// Roles per CTA (256 threads): warps 0-3 compute (thread r owns tensor-memory
-// lane r: a key row in dK/dV, a query row in dQ), warp 4 TMA producer, warp 5
-// MMA issuer (one elected thread; it also allocates tensor memory), warps 6-7
-// idle.  Tensor memory: S [0,128), dP [128,256), accumulators from 256; P and dS
+// Roles per CTA (384 threads): warps 0-7 compute in two warpgroups that split
+// each block's columns (thread r of a warpgroup owns tensor-memory lane r: a key
+// row in dK/dV, a query row in dQ), warp 8 TMA producer, warp 9 MMA issuer (one
+// elected thread; it also allocates tensor memory), warps 10-11 idle.  Tensor memory: S [0,128), dP [128,256), accumulators from 256; P and dS
 // are written as 16-bit pairs over the first 64 columns of S and dP, which the
 // thread has already read.  Every wait is bounded.
 #include <cuda.h>
@@ -36,7 +36,6 @@
 namespace fa {
 namespace {
 
-constexpr int kBwdThreads = 256;
 constexpr float kBwdLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -130,9 +129,15 @@ __global__ void __launch_bounds__(256) bwd_dot_kernel(const BwdParams p) {
   }
 }
 
+// Both tile kernels run 384 threads: two compute warpgroups (warpgroup c takes
+// columns [64 c, 64 c + 64) of every 128 x 128 block for the block's 128 rows),
+// warp 8 TMA producer, warp 9 MMA issuer, warps 10-11 idle.
+constexpr int kWideThreads = 384;
+
 // One CTA per (128-key block kb, KV head hk, batch b).
+
 template <int D, bool BF16, bool ALIBI>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kWideThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmD,
@@ -167,6 +172,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* empty = bars + 3;
   uint64_t* s_full = bars + 5;
   uint64_t* p_full = bars + 6;
+  uint64_t* s_read = bars + 7;   // warpgroup 0 holds its S^T columns in registers
+  uint64_t* dp_read = bars + 8;  // ... and its dP^T columns
   uint64_t* done = bars + 9;
   uint64_t* drain = bars + 10;
   uint64_t* dp_full = bars + 11;
@@ -174,7 +181,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     mbar_init(fix_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(full + s, 1);
@@ -182,14 +189,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(ds_full, 4);
+    mbar_init(p_full, 8);   // one arrival per compute warp
+    mbar_init(ds_full, 8);
+    mbar_init(s_read, 4);   // the four warps of warpgroup 0
+    mbar_init(dp_read, 4);
     mbar_init(done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_holder, Cfg::kTmemCols);
     tmem_relinquish();
   }
@@ -199,7 +208,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tbase = *tmem_holder;
   const WaitCtx w{abort_flag, p.status, p.timeout_ns};
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ======================================================== TMA producer
     if (lane == 0 && n_iter > 0) {
       tma_prefetch_map(&tmQ);
@@ -238,7 +247,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ======================================================== MMA issuer
     if (lane == 0 && n_iter > 0) {
       constexpr uint32_t idesc_s = f16_idesc(BF16, 128, 128, false, false);
@@ -294,11 +303,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       wait_drain_bwd(drain, 0, p.timeout_ns);  // own MMAs complete before teardown
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ======================================================== compute
-    const int r = threadIdx.x;  // key row within the block = TMEM lane
+    const int cg = warp / 4;  // query-column half of every block
+    const int r = (warp % 4) * 32 + lane;  // key row within the block = TMEM lane
     const int k = k0 + r;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
     bool ok = true;
     for (int n = 0; n < n_iter; ++n) {
       const int s = n & 1;
@@ -312,62 +322,98 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         break;
       }
       tc_fence_after();
-      const float* lse2 = stat + s * 256;
-      const float* dd = lse2 + 128;
-      // phase 1: P^T (kept in fp32 registers), 16-bit copy over read columns of S^T
+      const float* lse2 = stat + s * 256 + cg * 64;
+      const float* dd = stat + s * 256 + 128 + cg * 64;
+      // phase 1: P^T of this half (fp32 in registers), 16-bit copy to columns
+      // [32 cg, 32 cg + 32), which hold S^T columns of warpgroup 0: warpgroup 1
+      // stores only once warpgroup 0 has its scores in registers
       const bool open = mg.tile_open(qb, k0);  // uniform: the whole tile is unmasked
-      const float4* lse4 = reinterpret_cast<const float4*>(lse2);
-      float pf[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {  // 32 query columns at a time
-        uint32_t sv[32];
-        tmem_ld32(tbase + c * 32 + lane_off, sv);
+      float pf[64];
+      {
+        uint32_t sv[64];
+        tmem_ld32(tbase + cg * 64 + lane_off, sv);
+        tmem_ld32(tbase + cg * 64 + 32 + lane_off, sv + 32);
         tmem_ld_wait(sv);
-        uint32_t pp[16];
+        tmem_ld_wait(sv + 32);
+        if (cg == 0) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_read);
+        }
+        const float4* lse4 = reinterpret_cast<const float4*>(lse2);
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 l4 = lse4[(c * 32 + e) / 4];  // one broadcast load, four columns
+        for (int e = 0; e < 64; e += 4) {
+          const float4 l4 = lse4[e / 4];  // one broadcast load, four columns
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int qi = c * 32 + e + u;
-            const int q = qb + qi;
+            const int q = qb + cg * 64 + e + u;
             float x = __uint_as_float(sv[e + u]) * p.scale_log2;
             if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
-            pf[qi] = (open || mg.allowed(q, k)) ? ex2(x - lv[u]) : 0.f;
+            pf[e + u] = (open || mg.allowed(q, k)) ? ex2(x - lv[u]) : 0.f;
           }
-          pp[e / 2] = pack2<BF16>(pf[c * 32 + e], pf[c * 32 + e + 1]);
-          pp[e / 2 + 1] = pack2<BF16>(pf[c * 32 + e + 2], pf[c * 32 + e + 3]);
         }
-        tmem_st16(tbase + c * 16 + lane_off, pp);
+      }
+      if (cg == 1) {
+        ok = wait_bounded(s_read, n & 1, w);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pp[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pp[e] = pack2<BF16>(pf[c * 32 + 2 * e], pf[c * 32 + 2 * e + 1]);
+        tmem_st16(tbase + cg * 32 + c * 16 + lane_off, pp);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      // phase 2: dS^T = P^T * (dP^T - D) over read columns of dP^T
+      // phase 2: dS^T = P^T * (dP^T - D), the same column split over dP^T
       ok = wait_bounded(dp_full, n & 1, w);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t dp[32];
-        tmem_ld32(tbase + 128 + c * 32 + lane_off, dp);
+      {
+        uint32_t dp[64];
+        tmem_ld32(tbase + 128 + cg * 64 + lane_off, dp);
+        tmem_ld32(tbase + 128 + cg * 64 + 32 + lane_off, dp + 32);
         tmem_ld_wait(dp);
+        tmem_ld_wait(dp + 32);
+        if (cg == 0) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dp_read);
+        }
+#pragma unroll
+        for (int e = 0; e < 64; e += 4) {
+          const float4 d4 = reinterpret_cast<const float4*>(dd)[e / 4];
+          pf[e] *= __uint_as_float(dp[e]) - d4.x;
+          pf[e + 1] *= __uint_as_float(dp[e + 1]) - d4.y;
+          pf[e + 2] *= __uint_as_float(dp[e + 2]) - d4.z;
+          pf[e + 3] *= __uint_as_float(dp[e + 3]) - d4.w;
+        }
+      }
+      if (cg == 1) {
+        ok = wait_bounded(dp_read, n & 1, w);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
         uint32_t ps[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const int qi = c * 32 + e;
-          const float4 d4 = reinterpret_cast<const float4*>(dd)[qi / 4];
-          ps[e / 2] = pack2<BF16>(pf[qi] * (__uint_as_float(dp[e]) - d4.x),
-                                  pf[qi + 1] * (__uint_as_float(dp[e + 1]) - d4.y));
-          ps[e / 2 + 1] = pack2<BF16>(pf[qi + 2] * (__uint_as_float(dp[e + 2]) - d4.z),
-                                      pf[qi + 3] * (__uint_as_float(dp[e + 3]) - d4.w));
-        }
-        tmem_st16(tbase + 128 + c * 16 + lane_off, ps);
+        for (int e = 0; e < 16; ++e) ps[e] = pack2<BF16>(pf[c * 32 + 2 * e], pf[c * 32 + 2 * e + 1]);
+        tmem_st16(tbase + 128 + cg * 32 + c * 16 + lane_off, ps);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -386,7 +432,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint16_t* dst = static_cast<uint16_t*>(which ? p.dk : p.dv) + ro;
         const float mul = which ? p.scale : 1.f;
 #pragma unroll 1
-        for (int c2 = 0; c2 < D / 32; ++c2) {
+        for (int c2 = cg * (D / 64); c2 < (cg + 1) * (D / 64); ++c2) {  // this half's columns
           uint32_t o[32];
           if (n_iter > 0) {
             tmem_ld32(tbase + 256 + which * D + c2 * 32 + lane_off, o);
@@ -411,7 +457,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tbase, Cfg::kTmemCols);
   }
@@ -419,7 +465,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // One CTA per (128-query block, head h, batch b).
 template <int D, bool BF16, bool ALIBI>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kWideThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const BwdParams p) {
@@ -452,25 +498,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* empty = bars + 3;
   uint64_t* s_full = bars + 5;
   uint64_t* p_full = bars + 6;
+  uint64_t* s_read = bars + 7;  // warpgroup 0 holds its S columns in registers
   uint64_t* done = bars + 9;
   uint64_t* drain = bars + 10;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     mbar_init(fix_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);   // one arrival per compute warp
+    mbar_init(s_read, 4);
     mbar_init(done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_holder, Cfg::kTmemCols);
     tmem_relinquish();
   }
@@ -480,7 +528,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tbase = *tmem_holder;
   const WaitCtx w{abort_flag, p.status, p.timeout_ns};
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ======================================================== TMA producer
     if (lane == 0 && n_blk > 0) {
       tma_prefetch_map(&tmQ);
@@ -514,7 +562,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ======================================================== MMA issuer
     if (lane == 0 && n_blk > 0) {
       constexpr uint32_t idesc_s = f16_idesc(BF16, 128, 128, false, false);
@@ -544,11 +592,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       wait_drain_bwd(drain, 0, p.timeout_ns);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ======================================================== compute
-    const int r = threadIdx.x;  // query row within the block = TMEM lane
+    const int cg = warp / 4;  // key-column half of every block
+    const int r = (warp % 4) * 32 + lane;  // query row within the block = TMEM lane
     const int q = q0 + r;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
     const int64_t idx = (static_cast<int64_t>(b) * p.H + h) * p.sq_pad + q;
     const float lse2 = (q < p.Sq) ? p.lse2[idx] : INFINITY;
     const float dd = (q < p.Sq) ? p.dvec[idx] : 0.f;
@@ -563,29 +612,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       tc_fence_after();
       const bool open = mg.tile_open(q0, kb);  // uniform: the whole tile is unmasked
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {  // 32 key columns at a time
-        uint32_t sv[32], dp[32];
-        tmem_ld32(tbase + c * 32 + lane_off, sv);
-        tmem_ld32(tbase + 128 + c * 32 + lane_off, dp);
-        tmem_ld_wait(sv);
-        tmem_ld_wait(dp);
-        uint32_t ps[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int k = kb + c * 32 + e + u;
-            float x = __uint_as_float(sv[e + u]) * p.scale_log2;
-            if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
-            const float pr = (open || mg.allowed(q, k)) ? ex2(x - lse2) : 0.f;
-            ds[u] = pr * (__uint_as_float(dp[e + u]) - dd);
-          }
-          ps[e / 2] = pack2<BF16>(ds[0], ds[1]);
-        }
-        tmem_st16(tbase + c * 16 + lane_off, ps);  // dS over read columns of S
+      // this half's 64 key columns of S and dP; dS goes to S columns [32 cg, 32 cg +
+      // 32), which hold scores of warpgroup 0: warpgroup 1 stores only once those
+      // are in warpgroup 0's registers
+      uint32_t sv[64], dp[64];
+      tmem_ld32(tbase + cg * 64 + lane_off, sv);
+      tmem_ld32(tbase + cg * 64 + 32 + lane_off, sv + 32);
+      tmem_ld32(tbase + 128 + cg * 64 + lane_off, dp);
+      tmem_ld32(tbase + 128 + cg * 64 + 32 + lane_off, dp + 32);
+      tmem_ld_wait(sv);
+      tmem_ld_wait(sv + 32);
+      tmem_ld_wait(dp);
+      tmem_ld_wait(dp + 32);
+      if (cg == 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_read);
       }
+      uint32_t ps[32];
+#pragma unroll
+      for (int e = 0; e < 64; e += 2) {
+        float ds[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int k = kb + cg * 64 + e + u;
+          float x = __uint_as_float(sv[e + u]) * p.scale_log2;
+          if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
+          const float pr = (open || mg.allowed(q, k)) ? ex2(x - lse2) : 0.f;
+          ds[u] = pr * (__uint_as_float(dp[e + u]) - dd);
+        }
+        ps[e / 2] = pack2<BF16>(ds[0], ds[1]);
+      }
+      if (cg == 1) {
+        ok = wait_bounded(s_read, it & 1, w);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      tmem_st16(tbase + cg * 32 + lane_off, ps);
+      tmem_st16(tbase + cg * 32 + 16 + lane_off, ps + 16);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -599,7 +666,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint16_t* dst = static_cast<uint16_t*>(p.dq) +
                       ((static_cast<int64_t>(b) * p.Sq + q) * p.H + h) * D;
 #pragma unroll 1
-      for (int c2 = 0; c2 < D / 32; ++c2) {
+      for (int c2 = cg * (D / 64); c2 < (cg + 1) * (D / 64); ++c2) {  // this half's columns
         uint32_t o[32];
         if (n_blk > 0) {
           tmem_ld32(tbase + 256 + c2 * 32 + lane_off, o);
@@ -624,7 +691,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tbase, Cfg::kTmemCols);
   }
@@ -648,10 +715,10 @@ cudaError_t launch_bwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const 
                                 Cfg::kSmemAlloc)) != cudaSuccess)
     return e;
   const dim3 gkv(p.Hkv, p.B, (p.Sk + 127) / 128);
-  kkv<<<gkv, kBwdThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, tl, td, p);
+  kkv<<<gkv, kWideThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, tl, td, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const dim3 gq(p.H, p.B, (p.Sq + 127) / 128);
-  kq<<<gq, kBwdThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
+  kq<<<gq, kWideThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError();
 }
 
