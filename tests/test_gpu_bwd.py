@@ -1,7 +1,7 @@
 """GPU parity of fa_bwd (dQ, dK, dV) against the fp64 backward oracle.
 
 The kernel is given the oracle's O (rounded to the input dtype) and LSE, so that
-only the backward's own arithmetic is judged.  Its rounding steps, with u the
+only the backward's own arithmetic is checked.  Its rounding steps, with u the
 unit roundoff of the input dtype (2^-11 fp16, 2^-8 bf16), give the per-element
 bound used here (doubled for the compounding of two roundings, plus a floor for
 fp32 accumulation and the approximate exp2):
