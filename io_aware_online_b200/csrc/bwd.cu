@@ -48,8 +48,9 @@ struct BwdCfg {
   static constexpr int kStage = 2 * kTileBytes;       // 2 stages x {A, B} streamed tiles
   static constexpr int kStat = kStage + 4 * kTileBytes;  // [2 slots][2][128] fp32
   static constexpr int kBarOff = kStat + 2 * 2 * 128 * 4;
-  // fix_full, full[2], empty[2], s_full, p_full, stat[2], done, drain, dp_full, ds_full
-  static constexpr int kNumBars = 13;
+  // fix_full, full[2], empty[2], s_full, p_full, s_read, dp_read, done, drain, dp_full,
+  // ds_full (dQ kernel: second s_read and p_full at 12 and 13)
+  static constexpr int kNumBars = 14;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   // room to align the base to 1 KiB; at least 116 KiB, so that one CTA fills an SM
@@ -463,7 +464,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   }
 }
 
-// One CTA per (128-query block, head h, batch b).
+// One CTA per (128-query block, head h, batch b).  Tensor memory: two S buffers
+// [0, 128) and [128, 256) used by alternate key blocks, dP [256, 384), dQ from 384.
+// In issue order the products run S(0), dP(0); per block j, once every compute warp
+// holds S(j) and dP(j) in registers: S(j+1) [into the other buffer], dP(j+1); then,
+// once dS(j) is written, dQ(j).  The math of block j overlaps the products of block
+// j+1, and no completion barrier runs two phases ahead of its waiters.
 template <int D, bool BF16, bool ALIBI>
 __global__ void __launch_bounds__(kWideThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -497,10 +503,14 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   uint64_t* full = bars + 1;
   uint64_t* empty = bars + 3;
   uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* s_read = bars + 7;  // warpgroup 0 holds its S columns in registers
+  // alternating pairs, by block parity: an arrival for block j+2 needs the other
+  // side to have finished block j, so neither runs two phases ahead of its waiter
+  uint64_t* p_full[2] = {bars + 6, bars + 12};   // dS of the block written
+  uint64_t* s_read[2] = {bars + 7, bars + 13};   // warpgroup 0 holds its S columns
+  uint64_t* dp_read = bars + 8;  // every compute warp holds its dP columns in registers
   uint64_t* done = bars + 9;
   uint64_t* drain = bars + 10;
+  uint64_t* dp_full = bars + 11;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -511,8 +521,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       mbar_init(empty + s, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 8);   // one arrival per compute warp
-    mbar_init(s_read, 4);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(p_full[x], 8);  // dS written: one arrival per compute warp
+      mbar_init(s_read[x], 4);  // the four warps of warpgroup 0
+    }
+    mbar_init(dp_full, 1);
+    mbar_init(dp_read, 8);
     mbar_init(done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -569,22 +583,39 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       constexpr uint32_t idesc_acc = f16_idesc(BF16, 128, D, false, true);
       const uint64_t dQk = sw128_desc(smem_u32(fixA), 16, 1024);
       const uint64_t dOk = sw128_desc(smem_u32(fixB), 16, 1024);
-      bool ok = wait_bounded(fix_full, 0, w);
+      auto st_k = [&](int s) { return smem_u32(stage + s * 2 * Cfg::kTileBytes); };
+      bool ok = wait_bounded(fix_full, 0, w) && wait_bounded(full, 0, w);
+      if (ok) {
+        tc_fence_after();
+        fwd_issue_qk<D>(tbase, dQk, sw128_desc(st_k(0), 16, 1024), idesc_s);   // S(0)
+        tc_commit(s_full);
+        fwd_issue_qk<D>(tbase + 256, dOk, sw128_desc(st_k(0) + Cfg::kTileBytes, 16, 1024),
+                        idesc_s);                                               // dP(0)
+        tc_commit(dp_full);
+      }
       for (int it = 0; it < n_blk && ok; ++it) {
         const int s = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        if (!(ok = wait_bounded(full + s, ph, w))) break;
-        tc_fence_after();
-        const uint32_t sk = smem_u32(stage + s * 2 * Cfg::kTileBytes);
-        const uint32_t sv = sk + Cfg::kTileBytes;
-        fwd_issue_qk<D>(tbase, dQk, sw128_desc(sk, 16, 1024), idesc_s);         // S
-        fwd_issue_qk<D>(tbase + 128, dOk, sw128_desc(sv, 16, 1024), idesc_s);   // dP
-        tc_commit(s_full);
-        if (!(ok = wait_bounded(p_full, it & 1, w))) break;
+        const bool more = it + 1 < n_blk;
+        // every compute warp has passed its waits on S(j) and dP(j) and holds dP(j):
+        // S(j+1) and dP(j+1) may complete now without running two phases ahead of
+        // those waits, and dP(j+1) may overwrite the dP columns
+        if (!(ok = wait_bounded(dp_read, it & 1, w))) break;
+        if (more) {
+          if (!(ok = wait_bounded(full + (s ^ 1), ((it + 1) >> 1) & 1, w))) break;
+          tc_fence_after();
+          // S(j+1) into the other buffer (its dS(j-1) was read by dQ(j-1), issued before)
+          fwd_issue_qk<D>(tbase + (s ^ 1) * 128, dQk, sw128_desc(st_k(s ^ 1), 16, 1024),
+                          idesc_s);
+          tc_commit(s_full);
+          fwd_issue_qk<D>(tbase + 256, dOk, sw128_desc(st_k(s ^ 1) + Cfg::kTileBytes, 16, 1024),
+                          idesc_s);                                             // dP(j+1)
+          tc_commit(dp_full);
+        }
+        if (!(ok = wait_bounded(p_full[s], (it >> 1) & 1, w))) break;
         tc_fence_after();
         // dQ += dS K_j: B = K_j MN-major (rows are keys, the head dim contiguous)
-        fwd_issue_pv<D>(tbase + 256, tbase, sw128_desc(sk, Cfg::kChunkBytes, 1024), idesc_acc,
-                        it > 0);
+        fwd_issue_pv<D>(tbase + 384, tbase + s * 128,
+                        sw128_desc(st_k(s), Cfg::kChunkBytes, 1024), idesc_acc, it > 0);
         tc_commit(empty + s);
       }
       if (ok) tc_commit(done);
@@ -605,29 +636,33 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     bool ok = true;
     for (int it = 0; it < n_blk; ++it) {
       const int kb = (j_lo + it) * 128;
-      ok = wait_bounded(s_full, it & 1, w);
+      ok = wait_bounded(s_full, it & 1, w) && wait_bounded(dp_full, it & 1, w);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      const uint32_t tS = tbase + (it & 1) * 128;  // this block's S buffer
       const bool open = mg.tile_open(q0, kb);  // uniform: the whole tile is unmasked
       // this half's 64 key columns of S and dP; dS goes to S columns [32 cg, 32 cg +
       // 32), which hold scores of warpgroup 0: warpgroup 1 stores only once those
       // are in warpgroup 0's registers
       uint32_t sv[64], dp[64];
-      tmem_ld32(tbase + cg * 64 + lane_off, sv);
-      tmem_ld32(tbase + cg * 64 + 32 + lane_off, sv + 32);
-      tmem_ld32(tbase + 128 + cg * 64 + lane_off, dp);
-      tmem_ld32(tbase + 128 + cg * 64 + 32 + lane_off, dp + 32);
+      tmem_ld32(tS + cg * 64 + lane_off, sv);
+      tmem_ld32(tS + cg * 64 + 32 + lane_off, sv + 32);
+      tmem_ld32(tbase + 256 + cg * 64 + lane_off, dp);
+      tmem_ld32(tbase + 256 + cg * 64 + 32 + lane_off, dp + 32);
       tmem_ld_wait(sv);
       tmem_ld_wait(sv + 32);
       tmem_ld_wait(dp);
       tmem_ld_wait(dp + 32);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dp_read);  // dP(j+1) may overwrite the dP columns
       if (cg == 0) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_read);
+        if (lane == 0) mbar_arrive(s_read[it & 1]);
       }
       uint32_t ps[32];
 #pragma unroll
@@ -644,19 +679,19 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         ps[e / 2] = pack2<BF16>(ds[0], ds[1]);
       }
       if (cg == 1) {
-        ok = wait_bounded(s_read, it & 1, w);
+        ok = wait_bounded(s_read[it & 1], (it >> 1) & 1, w);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
         }
         tc_fence_after();
       }
-      tmem_st16(tbase + cg * 32 + lane_off, ps);
-      tmem_st16(tbase + cg * 32 + 16 + lane_off, ps + 16);
+      tmem_st16(tS + cg * 32 + lane_off, ps);
+      tmem_st16(tS + cg * 32 + 16 + lane_off, ps + 16);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full[it & 1]);
     }
     // ---- epilogue: scale * dQ -> 16-bit
     if (ok && n_blk > 0) ok = wait_bounded(done, 0, w);
@@ -669,7 +704,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       for (int c2 = cg * (D / 64); c2 < (cg + 1) * (D / 64); ++c2) {  // this half's columns
         uint32_t o[32];
         if (n_blk > 0) {
-          tmem_ld32(tbase + 256 + c2 * 32 + lane_off, o);
+          tmem_ld32(tbase + 384 + c2 * 32 + lane_off, o);
           tmem_ld_wait(o);
         } else {
 #pragma unroll
