@@ -396,6 +396,74 @@ def run_bwd(args, rank, world, local):
             "gpu_launches": 3 * K, "clocks": clk.summary()}
 
 
+# TFLOPS vs sequence length of the causal prefill (B=4, H=Hkv=32)
+SWEEP = dict(B=4, H=32, d=(64, 128), S=(512, 1024, 2048, 4096, 8192, 16384),
+             dtype=("fp16", "bf16"))
+
+
+def run_sweep(args, rank, world, local):
+    """--only sweep: the causal prefill's TFLOPS over head dims, sequence lengths
+    and 16-bit types; one JSON line whose value is the largest point (d=128,
+    S=16384, bf16) and whose ``curve`` holds every point."""
+    import io_aware_online_b200 as fa
+    from io_aware_online_b200 import build as fa_build
+    fa_build.build()
+    fa.load()
+    dev = torch.device("cuda", local)
+    _, tflops_peak, peak_src = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    c = SWEEP
+    K = min(args.steps, 10)
+    curve = []
+    with Clocks(dev.index if dev.index is not None else 0) as clk:
+        for d in c["d"]:
+            for S in c["S"]:
+                for dname in c["dtype"]:
+                    dt = synth.DTYPES[dname]
+                    gen = torch.Generator(device=dev).manual_seed(3300 + S + d + rank)
+                    shp = (c["B"], S, c["H"], d)
+                    q, k, v = (torch.randn(shp, generator=gen, device=dev).to(dt)
+                               for _ in range(3))
+                    out = torch.empty_like(q)
+                    lse = torch.empty((c["B"], c["H"], S), dtype=torch.float32, device=dev)
+                    for _ in range(args.warmup):
+                        flush.zero_()
+                        fa.fa_fwd(q, k, v, out=out, lse=lse, causal=True, stream=stream)
+                    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                          for _ in range(K)]
+                    barrier(world)
+                    torch.cuda.synchronize(dev)
+                    for i in range(K):
+                        flush.zero_()
+                        ev[i][0].record(stream)
+                        fa.fa_fwd(q, k, v, out=out, lse=lse, causal=True, stream=stream)
+                        ev[i][1].record(stream)
+                    torch.cuda.synchronize(dev)
+                    barrier(world)
+                    ms = max_over_ranks(statistics.median(e[0].elapsed_time(e[1]) for e in ev),
+                                        world)
+                    tf = 4.0 * d * c["B"] * c["H"] * causal_pairs(S, S) / (ms * 1e-3) / 1e12
+                    curve.append({"d": d, "S": S, "dtype": dname, "ms": round(ms, 4),
+                                  "tflops": round(tf, 1), "frac": round(tf / tflops_peak, 4)})
+                    del q, k, v, out, lse
+    assert fa.fa_device_status(clear=True) == 0, "device status flags raised during the sweep"
+    top = curve[-1]
+    return {"metric": "attn fwd TFLOPS vs seqlen (causal prefill)",
+            "value": round(top["tflops"] * world, 2), "unit": "TFLOPS", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": top["ms"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp16 / bf16; fp32 accumulate", "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": "causal prefill sweep B=4 H=32 over d, S and dtype; value = "
+                                   "d=128 S=16384 bf16", "B": c["B"], "H": c["H"],
+                       "l2": "flushed between launches (256 MiB write, untimed)",
+                       "parallelism": f"dp{world} (independent replicas)"},
+            "roofline": {"bound": "tensor", "achieved": top["tflops"], "peak": tflops_peak,
+                         "unit": "TFLOP/s", "frac": top["frac"], "traffic": None,
+                         "kernel": "fwd_kernel<128, bf16, causal>", "peak_source": peak_src},
+            "curve": curve, "gpu_launches": K * len(curve), "clocks": clk.summary()}
+
+
 def run_fp8(args, rank, world, local):
     """--only fp8: time fa_fwd_fp8 on the d=128 causal prefill workload."""
     import io_aware_online_b200 as fa
@@ -625,7 +693,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "chunked", "append", "fp8",
-                                       "bwd"],
+                                       "bwd", "sweep"],
                     default="all",
                     help="time one part of the step (profiling / sweeps), or one of the "
                          "cache-update rows on its own workload (chunked, append)")
@@ -644,8 +712,9 @@ def main():
             if rank == 0:
                 print(json.dumps(run_reference(args, rank, world)), flush=True)
             return
-        if args.only in ("chunked", "append", "fp8", "bwd"):
-            fn = {"fp8": run_fp8, "bwd": run_bwd}.get(args.only, run_cache_rows)
+        if args.only in ("chunked", "append", "fp8", "bwd", "sweep"):
+            fn = {"fp8": run_fp8, "bwd": run_bwd, "sweep": run_sweep}.get(args.only,
+                                                                          run_cache_rows)
             res = fn(args, rank, world, local)
             if rank == 0:
                 print(json.dumps(res), flush=True)
