@@ -65,12 +65,10 @@ struct BwdCfg {
 struct MaskGeo {
   int off, Sk, Sq, wl, right;
   bool has_left, has_right;
+  // branch-free, so that a masked tile's loop stays one basic block
   __device__ __forceinline__ bool allowed(int i, int j) const {
-    if (i >= Sq || j >= Sk) return false;
     const int c = i + off;
-    if (has_right && j > c + right) return false;
-    if (has_left && j < c - wl) return false;
-    return true;
+    return (i < Sq) & (j < Sk) & (!has_right | (j <= c + right)) & (!has_left | (j >= c - wl));
   }
   // every (query, key) of the 128 x 128 tile at (i0, j0) allowed: no mask needed
   __device__ __forceinline__ bool tile_open(int i0, int j0) const {
@@ -134,6 +132,11 @@ __global__ void __launch_bounds__(256) bwd_dot_kernel(const BwdParams p) {
 // columns [64 c, 64 c + 64) of every 128 x 128 block for the block's 128 rows),
 // warp 8 TMA producer, warp 9 MMA issuer, warps 10-11 idle.
 constexpr int kWideThreads = 384;
+// registers per thread: 168 at launch (one CTA per SM); the compute warpgroups
+// take what the producer, the MMA issuer and the idle warps do not need
+constexpr uint32_t kBwdLaunchRegs = 168, kBwdComputeRegs = 208, kBwdOtherRegs = 88;
+static_assert(256 * kBwdComputeRegs + 128 * kBwdOtherRegs == kWideThreads * kBwdLaunchRegs,
+              "register re-split must add up to the launch registers");
 
 // One CTA per (128-key block kb, KV head hk, batch b).
 
@@ -209,7 +212,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   const uint32_t tbase = *tmem_holder;
   const WaitCtx w{abort_flag, p.status, p.timeout_ns};
 
-  if (warp == 8) {
+  // register re-split inside the role branches (a merge of the two limits before
+  // them would hold all later code to the smaller one)
+  if (warp >= 8) {
+   regs_dec<kBwdOtherRegs>();
+   if (warp == 8) {
     // ======================================================== TMA producer
     if (lane == 0 && n_iter > 0) {
       tma_prefetch_map(&tmQ);
@@ -248,7 +255,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+   } else if (warp == 9) {
     // ======================================================== MMA issuer
     if (lane == 0 && n_iter > 0) {
       constexpr uint32_t idesc_s = f16_idesc(BF16, 128, 128, false, false);
@@ -304,7 +311,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       wait_drain_bwd(drain, 0, p.timeout_ns);  // own MMAs complete before teardown
     }
     __syncwarp();
-  } else if (warp < 8) {
+   }
+  } else {
+    regs_inc<kBwdComputeRegs>();
     // ======================================================== compute
     const int cg = warp / 4;  // query-column half of every block
     const int r = (warp % 4) * 32 + lane;  // key row within the block = TMEM lane
@@ -342,18 +351,29 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           if (lane == 0) mbar_arrive(s_read);
         }
         const float4* lse4 = reinterpret_cast<const float4*>(lse2);
+        // every exponential is taken and a masked one then dropped by a select: a
+        // branch per element would split the loop into blocks of one exponential
+        // each and expose the whole latency of every one
+        auto probs = [&](auto masked_t) {
+          constexpr bool kMasked = decltype(masked_t)::value;
 #pragma unroll
-        for (int e = 0; e < 64; e += 4) {
-          const float4 l4 = lse4[e / 4];  // one broadcast load, four columns
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          for (int e = 0; e < 64; e += 4) {
+            const float4 l4 = lse4[e / 4];  // one broadcast load, four columns
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int q = qb + cg * 64 + e + u;
-            float x = __uint_as_float(sv[e + u]) * p.scale_log2;
-            if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
-            pf[e + u] = (open || mg.allowed(q, k)) ? ex2(x - lv[u]) : 0.f;
+            for (int u = 0; u < 4; ++u) {
+              const int q = qb + cg * 64 + e + u;
+              float x = __uint_as_float(sv[e + u]) * p.scale_log2;
+              if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
+              const float ev = ex2(x - lv[u]);
+              pf[e + u] = (!kMasked || mg.allowed(q, k)) ? ev : 0.f;
+            }
           }
-        }
+        };
+        if (open)
+          probs(std::false_type{});
+        else
+          probs(std::true_type{});
       }
       if (cg == 1) {
         ok = wait_bounded(s_read, n & 1, w);
@@ -542,7 +562,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   const uint32_t tbase = *tmem_holder;
   const WaitCtx w{abort_flag, p.status, p.timeout_ns};
 
-  if (warp == 8) {
+  // register re-split inside the role branches (a merge of the two limits before
+  // them would hold all later code to the smaller one)
+  if (warp >= 8) {
+   regs_dec<kBwdOtherRegs>();
+   if (warp == 8) {
     // ======================================================== TMA producer
     if (lane == 0 && n_blk > 0) {
       tma_prefetch_map(&tmQ);
@@ -576,7 +600,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+   } else if (warp == 9) {
     // ======================================================== MMA issuer
     if (lane == 0 && n_blk > 0) {
       constexpr uint32_t idesc_s = f16_idesc(BF16, 128, 128, false, false);
@@ -623,7 +647,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       wait_drain_bwd(drain, 0, p.timeout_ns);
     }
     __syncwarp();
-  } else if (warp < 8) {
+   }
+  } else {
+    regs_inc<kBwdComputeRegs>();
     // ======================================================== compute
     const int cg = warp / 4;  // key-column half of every block
     const int r = (warp % 4) * 32 + lane;  // query row within the block = TMEM lane
@@ -664,20 +690,29 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(s_read[it & 1]);
       }
+      // every exponential is taken, a masked one then dropped by a select (no
+      // branch per element: the loop stays one block the scheduler can overlap)
       uint32_t ps[32];
+      auto grads = [&](auto masked_t) {
+        constexpr bool kMasked = decltype(masked_t)::value;
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {
-        float ds[2];
+        for (int e = 0; e < 64; e += 2) {
+          float ds[2];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int k = kb + cg * 64 + e + u;
-          float x = __uint_as_float(sv[e + u]) * p.scale_log2;
-          if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
-          const float pr = (open || mg.allowed(q, k)) ? ex2(x - lse2) : 0.f;
-          ds[u] = pr * (__uint_as_float(dp[e + u]) - dd);
+          for (int u = 0; u < 2; ++u) {
+            const int k = kb + cg * 64 + e + u;
+            float x = __uint_as_float(sv[e + u]) * p.scale_log2;
+            if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
+            const float g = ex2(x - lse2) * (__uint_as_float(dp[e + u]) - dd);
+            ds[u] = (!kMasked || mg.allowed(q, k)) ? g : 0.f;
+          }
+          ps[e / 2] = pack2<BF16>(ds[0], ds[1]);
         }
-        ps[e / 2] = pack2<BF16>(ds[0], ds[1]);
-      }
+      };
+      if (open)
+        grads(std::false_type{});
+      else
+        grads(std::true_type{});
       if (cg == 1) {
         ok = wait_bounded(s_read[it & 1], (it >> 1) & 1, w);
         if (!__all_sync(0xffffffffu, ok)) {
