@@ -354,20 +354,31 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         // every exponential is taken and a masked one then dropped by a select: a
         // branch per element would split the loop into blocks of one exponential
         // each and expose the whole latency of every one
+        // one pair in four is evaluated on the FMA pipe (exp2_fma2), the rest on MUFU
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
         auto probs = [&](auto masked_t) {
           constexpr bool kMasked = decltype(masked_t)::value;
 #pragma unroll
           for (int e = 0; e < 64; e += 4) {
             const float4 l4 = lse4[e / 4];  // one broadcast load, four columns
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+            float2 a[2] = {
+                fma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2,
+                     make_float2(-l4.x, -l4.y)),
+                fma2(make_float2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), sc2,
+                     make_float2(-l4.z, -l4.w))};
+            if constexpr (ALIBI) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int q = qb + cg * 64 + e + u;
-              float x = __uint_as_float(sv[e + u]) * p.scale_log2;
-              if constexpr (ALIBI) x = fmaf(-slope2, fabsf(static_cast<float>(q + mg.off - k)), x);
-              const float ev = ex2(x - lv[u]);
-              pf[e + u] = (!kMasked || mg.allowed(q, k)) ? ev : 0.f;
+              for (int u = 0; u < 4; ++u) {
+                const float bias = -slope2 * fabsf(static_cast<float>(qb + cg * 64 + e + u + mg.off - k));
+                if (u % 2 == 0) a[u / 2].x += bias; else a[u / 2].y += bias;
+              }
             }
+            const float2 e0 = (e % 8 == 0) ? exp2_fma2(a[0]) : make_float2(ex2(a[0].x), ex2(a[0].y));
+            const float2 e1 = make_float2(ex2(a[1].x), ex2(a[1].y));
+            const float ev[4] = {e0.x, e0.y, e1.x, e1.y};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              pf[e + u] = (!kMasked || mg.allowed(qb + cg * 64 + e + u, k)) ? ev[u] : 0.f;
           }
         };
         if (open)
