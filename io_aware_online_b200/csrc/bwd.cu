@@ -38,19 +38,21 @@ namespace {
 
 constexpr float kBwdLog2e = 1.4426950408889634f;
 
+// Shared memory of the dK/dV kernel: K_j and V_j, a two-stage ring of {Q_i, dO_i}
+// and the column statistics of each stage.
 template <int D>
 struct BwdCfg {
   static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms per row
   static constexpr int kTileBytes = 128 * D * 2;      // one 128-row tile
   static constexpr int kChunkBytes = 128 * 128;
-  static constexpr int kFixA = 0;                     // K_j (dK/dV) or Q_i (dQ)
-  static constexpr int kFixB = kTileBytes;            // V_j (dK/dV) or dO_i (dQ)
-  static constexpr int kStage = 2 * kTileBytes;       // 2 stages x {A, B} streamed tiles
+  static constexpr int kFixA = 0;                     // K_j
+  static constexpr int kFixB = kTileBytes;            // V_j
+  static constexpr int kStage = 2 * kTileBytes;       // 2 stages x {Q_i, dO_i}
   static constexpr int kStat = kStage + 4 * kTileBytes;  // [2 slots][2][128] fp32
   static constexpr int kBarOff = kStat + 2 * 2 * 128 * 4;
   // fix_full, full[2], empty[2], s_full, p_full, s_read, dp_read, done, drain, dp_full,
-  // ds_full (dQ kernel: second s_read and p_full at 12 and 13)
-  static constexpr int kNumBars = 14;
+  // ds_full
+  static constexpr int kNumBars = 13;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   // room to align the base to 1 KiB; at least 116 KiB, so that one CTA fills an SM
@@ -58,7 +60,32 @@ struct BwdCfg {
   // allocation for the first to finish)
   static constexpr int kSmemAlloc =
       (kSmemBytes + 1024 > 116 * 1024) ? kSmemBytes + 1024 : 116 * 1024;
-  static constexpr int kTmemCols = 512;                 // S 128 + dP 128 + up to 2 x D
+  static constexpr int kTmemCols = 512;                 // S^T 128 + dP^T 128 + 2 x D
+};
+
+// Shared memory of the dQ kernel: Q_i and dO_i, then separate rings of K_j (three
+// stages: K_j is read until dQ(j)) and V_j (two stages: V_j is released once dP(j)
+// has run), so that the tiles of block j+1 arrive while block j is processed.
+template <int D>
+struct DqCfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kChunkBytes = 128 * 128;
+  static constexpr int kKStages = 3, kVStages = 2;
+  static constexpr int kFixA = 0;                      // Q_i
+  static constexpr int kFixB = kTileBytes;             // dO_i
+  static constexpr int kK = 2 * kTileBytes;
+  static constexpr int kV = kK + kKStages * kTileBytes;
+  static constexpr int kBarOff = kV + kVStages * kTileBytes;
+  // fix_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, p_full[2],
+  // s_read[2], dp_read, done, drain, dp_full
+  static constexpr int kNumBars = 20;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16;
+  static constexpr int kSmemAlloc =
+      (kSmemBytes + 1024 > 116 * 1024) ? kSmemBytes + 1024 : 116 * 1024;
+  static_assert(kSmemAlloc <= 227 * 1024, "dQ tiles exceed shared memory");
+  static constexpr int kTmemCols = 512;                // S 2 x 128 + dP 128 + dQ <= 128
 };
 
 // Key j allowed for query i (bottom-right alignment, off = Sk - Sq).
@@ -99,25 +126,32 @@ __device__ __forceinline__ bool wait_drain_bwd(uint64_t* bar, uint32_t parity, u
   return true;
 }
 
-// D[b, h, i] = sum_c dO[b, i, h, c] * O[b, i, h, c], fp32; one warp per row.
+// D[b, h, i] = sum_c dO[b, i, h, c] * O[b, i, h, c], fp32.  16-byte loads: a row is
+// D / 8 lanes (16 at d = 128, 8 at d = 64), a warp takes 32 / (D / 8) rows.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) bwd_dot_kernel(const BwdParams p) {
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + threadIdx.x / 32;  // (b, i, h)
+  constexpr int kLanes = D / 8;
+  constexpr int kRowsPerWarp = 32 / kLanes;
   const int lane = threadIdx.x % 32;
-  if (row >= static_cast<int64_t>(p.B) * p.Sq * p.H) return;
-  constexpr int kPer = D / 32;  // elements per lane: 2 or 4
-  const uint16_t* o = static_cast<const uint16_t*>(p.out) + row * D + lane * kPer;
-  const uint16_t* g = static_cast<const uint16_t*>(p.dout) + row * D + lane * kPer;
+  const int l = lane % kLanes;
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * 8 + threadIdx.x / 32) * kRowsPerWarp +
+                      lane / kLanes;  // (b, i, h)
+  const bool live = row < static_cast<int64_t>(p.B) * p.Sq * p.H;
   float acc = 0.f;
+  if (live) {
+    const uint4 o = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.out) + row * D + l * 8);
+    const uint4 g = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + row * D + l * 8);
+    const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
-  for (int e = 0; e < kPer; e += 2) {
-    const float2 a = unpack2<BF16>(*reinterpret_cast<const uint32_t*>(o + e));
-    const float2 c = unpack2<BF16>(*reinterpret_cast<const uint32_t*>(g + e));
-    acc = fmaf(a.x, c.x, fmaf(a.y, c.y, acc));
+    for (int e = 0; e < 4; ++e) {
+      const float2 a = unpack2<BF16>(ow[e]);
+      const float2 c = unpack2<BF16>(gw[e]);
+      acc = fmaf(a.x, c.x, fmaf(a.y, c.y, acc));
+    }
   }
 #pragma unroll
-  for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-  if (lane == 0) {
+  for (int m = kLanes / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if (live && l == 0) {
     const int h = static_cast<int>(row % p.H);
     const int64_t bi = row / p.H;  // b * Sq + i
     const int i = static_cast<int>(bi % p.Sq);
@@ -506,7 +540,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const BwdParams p) {
-  using Cfg = BwdCfg<D>;
+  using Cfg = DqCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -526,30 +560,39 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   const int j_lo = k_begin / 128;
   const int n_blk = (q0 < p.Sq && k_end > k_begin) ? (k_end + 127) / 128 - j_lo : 0;
 
+  constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages;
   uint8_t* fixA = smem + Cfg::kFixA;  // Q_i
   uint8_t* fixB = smem + Cfg::kFixB;  // dO_i
-  uint8_t* stage = smem + Cfg::kStage;  // slot s: K_j at s * 2 tiles, V_j after it
+  uint8_t* ring_k = smem + Cfg::kK;   // K_j in stage j % KS
+  uint8_t* ring_v = smem + Cfg::kV;   // V_j in stage j % VS
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
   uint64_t* fix_full = bars;
-  uint64_t* full = bars + 1;
-  uint64_t* empty = bars + 3;
-  uint64_t* s_full = bars + 5;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 1 + KS;
+  uint64_t* v_full = bars + 1 + 2 * KS;
+  uint64_t* v_empty = bars + 1 + 2 * KS + VS;
+  uint64_t* s_full = bars + 1 + 2 * KS + 2 * VS;
   // alternating pairs, by block parity: an arrival for block j+2 needs the other
   // side to have finished block j, so neither runs two phases ahead of its waiter
-  uint64_t* p_full[2] = {bars + 6, bars + 12};   // dS of the block written
-  uint64_t* s_read[2] = {bars + 7, bars + 13};   // warpgroup 0 holds its S columns
-  uint64_t* dp_read = bars + 8;  // every compute warp holds its dP columns in registers
-  uint64_t* done = bars + 9;
-  uint64_t* drain = bars + 10;
-  uint64_t* dp_full = bars + 11;
+  uint64_t* p_full[2] = {s_full + 1, s_full + 2};   // dS of the block written
+  uint64_t* s_read[2] = {s_full + 3, s_full + 4};   // warpgroup 0 holds its S columns
+  uint64_t* dp_read = s_full + 5;  // every compute warp holds its dP columns in registers
+  uint64_t* done = s_full + 6;
+  uint64_t* drain = s_full + 7;
+  uint64_t* dp_full = s_full + 8;
+  static_assert(1 + 2 * KS + 2 * VS + 9 == Cfg::kNumBars, "barrier count");
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
   if (warp == 8 && lane == 0) {
     mbar_init(fix_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(empty + s, 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
     }
     mbar_init(s_full, 1);
     for (int x = 0; x < 2; ++x) {
@@ -589,25 +632,32 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         tma_load_4d(fixA + c * Cfg::kChunkBytes, &tmQ, fix_full, c * 64, q0, h, b);
         tma_load_4d(fixB + c * Cfg::kChunkBytes, &tmDO, fix_full, c * 64, q0, h, b);
       }
-      int last[2] = {-1, -1};
+      int last_k[KS], last_v[VS];
+      for (int s = 0; s < KS; ++s) last_k[s] = -1;
+      for (int s = 0; s < VS; ++s) last_v[s] = -1;
       for (int it = 0; it < n_blk; ++it) {
-        const int s = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
+        const int sk = it % KS, sv = it % VS;
+        const uint32_t phk = (it / KS) & 1, phv = (it / VS) & 1;
         const int kb = (j_lo + it) * 128;
-        if (!wait_bounded(empty + s, ph ^ 1, w)) break;
-        mbar_arrive_expect_tx(full + s, 2 * Cfg::kTileBytes);
-        uint8_t* st = stage + s * 2 * Cfg::kTileBytes;
-        for (int c = 0; c < Cfg::kChunks; ++c) {
-          tma_load_4d(st + c * Cfg::kChunkBytes, &tmK, full + s, c * 64, kb, hk, b);
-          tma_load_4d(st + Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmV, full + s, c * 64, kb, hk,
-                      b);
-        }
-        last[s] = ph;
+        if (!wait_bounded(k_empty + sk, phk ^ 1, w)) break;
+        mbar_arrive_expect_tx(k_full + sk, Cfg::kTileBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_4d(ring_k + sk * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmK, k_full + sk,
+                      c * 64, kb, hk, b);
+        last_k[sk] = phk;
+        if (!wait_bounded(v_empty + sv, phv ^ 1, w)) break;
+        mbar_arrive_expect_tx(v_full + sv, Cfg::kTileBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_4d(ring_v + sv * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmV, v_full + sv,
+                      c * 64, kb, hk, b);
+        last_v[sv] = phv;
       }
       if (*abort_flag) {
         wait_drain_bwd(fix_full, 0, p.timeout_ns);
-        for (int s = 0; s < 2; ++s)
-          if (last[s] >= 0) wait_drain_bwd(full + s, last[s], p.timeout_ns);
+        for (int s = 0; s < KS; ++s)
+          if (last_k[s] >= 0) wait_drain_bwd(k_full + s, last_k[s], p.timeout_ns);
+        for (int s = 0; s < VS; ++s)
+          if (last_v[s] >= 0) wait_drain_bwd(v_full + s, last_v[s], p.timeout_ns);
       }
     }
     __syncwarp();
@@ -618,15 +668,17 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       constexpr uint32_t idesc_acc = f16_idesc(BF16, 128, D, false, true);
       const uint64_t dQk = sw128_desc(smem_u32(fixA), 16, 1024);
       const uint64_t dOk = sw128_desc(smem_u32(fixB), 16, 1024);
-      auto st_k = [&](int s) { return smem_u32(stage + s * 2 * Cfg::kTileBytes); };
-      bool ok = wait_bounded(fix_full, 0, w) && wait_bounded(full, 0, w);
+      auto st_k = [&](int it) { return smem_u32(ring_k + (it % KS) * Cfg::kTileBytes); };
+      auto st_v = [&](int it) { return smem_u32(ring_v + (it % VS) * Cfg::kTileBytes); };
+      bool ok = wait_bounded(fix_full, 0, w) && wait_bounded(k_full, 0, w) &&
+                wait_bounded(v_full, 0, w);
       if (ok) {
         tc_fence_after();
         fwd_issue_qk<D>(tbase, dQk, sw128_desc(st_k(0), 16, 1024), idesc_s);   // S(0)
         tc_commit(s_full);
-        fwd_issue_qk<D>(tbase + 256, dOk, sw128_desc(st_k(0) + Cfg::kTileBytes, 16, 1024),
-                        idesc_s);                                               // dP(0)
+        fwd_issue_qk<D>(tbase + 256, dOk, sw128_desc(st_v(0), 16, 1024), idesc_s);  // dP(0)
         tc_commit(dp_full);
+        tc_commit(v_empty);  // V_0 is read by dP(0) alone
       }
       for (int it = 0; it < n_blk && ok; ++it) {
         const int s = it & 1;
@@ -636,22 +688,24 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         // those waits, and dP(j+1) may overwrite the dP columns
         if (!(ok = wait_bounded(dp_read, it & 1, w))) break;
         if (more) {
-          if (!(ok = wait_bounded(full + (s ^ 1), ((it + 1) >> 1) & 1, w))) break;
+          const int n1 = it + 1;
+          if (!(ok = wait_bounded(k_full + n1 % KS, (n1 / KS) & 1, w))) break;
           tc_fence_after();
           // S(j+1) into the other buffer (its dS(j-1) was read by dQ(j-1), issued before)
-          fwd_issue_qk<D>(tbase + (s ^ 1) * 128, dQk, sw128_desc(st_k(s ^ 1), 16, 1024),
-                          idesc_s);
+          fwd_issue_qk<D>(tbase + (s ^ 1) * 128, dQk, sw128_desc(st_k(n1), 16, 1024), idesc_s);
           tc_commit(s_full);
-          fwd_issue_qk<D>(tbase + 256, dOk, sw128_desc(st_k(s ^ 1) + Cfg::kTileBytes, 16, 1024),
-                          idesc_s);                                             // dP(j+1)
+          if (!(ok = wait_bounded(v_full + n1 % VS, (n1 / VS) & 1, w))) break;
+          tc_fence_after();
+          fwd_issue_qk<D>(tbase + 256, dOk, sw128_desc(st_v(n1), 16, 1024), idesc_s);  // dP(j+1)
           tc_commit(dp_full);
+          tc_commit(v_empty + n1 % VS);
         }
         if (!(ok = wait_bounded(p_full[s], (it >> 1) & 1, w))) break;
         tc_fence_after();
         // dQ += dS K_j: B = K_j MN-major (rows are keys, the head dim contiguous)
         fwd_issue_pv<D>(tbase + 384, tbase + s * 128,
-                        sw128_desc(st_k(s), Cfg::kChunkBytes, 1024), idesc_acc, it > 0);
-        tc_commit(empty + s);
+                        sw128_desc(st_k(it), Cfg::kChunkBytes, 1024), idesc_acc, it > 0);
+        tc_commit(k_empty + it % KS);
       }
       if (ok) tc_commit(done);
       tc_commit(drain);
@@ -784,7 +838,9 @@ cudaError_t launch_bwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const BwdParams& p, cudaStream_t stream) {
   using Cfg = BwdCfg<D>;
   const int64_t rows = static_cast<int64_t>(p.B) * p.Sq * p.H;
-  bwd_dot_kernel<D, BF16><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
+  constexpr int kRowsPerBlock = 8 * (32 / (D / 8));
+  bwd_dot_kernel<D, BF16><<<static_cast<unsigned>((rows + kRowsPerBlock - 1) / kRowsPerBlock), 256,
+                            0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   auto kkv = bwd_dkdv_kernel<D, BF16, ALIBI>;
@@ -793,13 +849,13 @@ cudaError_t launch_bwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const 
                                 Cfg::kSmemAlloc)) != cudaSuccess)
     return e;
   if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Cfg::kSmemAlloc)) != cudaSuccess)
+                                DqCfg<D>::kSmemAlloc)) != cudaSuccess)
     return e;
   const dim3 gkv(p.Hkv, p.B, (p.Sk + 127) / 128);
   kkv<<<gkv, kWideThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, tl, td, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const dim3 gq(p.H, p.B, (p.Sq + 127) / 128);
-  kq<<<gq, kWideThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
+  kq<<<gq, kWideThreads, DqCfg<D>::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError();
 }
 
