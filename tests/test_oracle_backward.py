@@ -31,8 +31,11 @@ def loss_grads_fd(q, k, v, do, h=1e-6, **kw):
 
 
 @pytest.mark.parametrize("kw", [dict(), dict(causal=True), dict(causal=True, window=(2, -1)),
-                                dict(window=(1, 1))],
-                         ids=["plain", "causal", "causal-window", "window"])
+                                dict(window=(1, 1)),
+                                dict(causal=True, alibi_slopes=np.array([0.5, 0.125])),
+                                dict(alibi_slopes=np.array([0.25, 1.0]), scale=0.7)],
+                         ids=["plain", "causal", "causal-window", "window", "causal-alibi",
+                              "alibi-scale"])
 def test_backward_matches_finite_differences(kw):
     rng = np.random.default_rng(7)
     B, Sq, Sk, H, Hkv, d = 1, 4, 6, 2, 1, 3
