@@ -189,3 +189,50 @@ def test_fp8_validation(lib):
     assert f8(d=64) == FA_ERR_UNSUPPORTED
     assert f8(qd=0.0) == FA_ERR_INVALID_ARG
     assert f8(vd=float("inf")) == FA_ERR_INVALID_ARG
+
+
+def bwd(lib, **kw):
+    a = dict(dout=P, q=P, k=P, v=P, out=P, lse=P, dq=P, dk=P, dv=P, dtype=1, B=1, Sq=256, Sk=256,
+             H=2, Hkv=2, d=128, scale=float("nan"), causal=1, wl=-1, wr=-1, softcap=0.0,
+             alibi=None, ws=P, ws_bytes=None, stream=None)
+    a.update(kw)
+    if a["ws_bytes"] is None:
+        a["ws_bytes"] = lib.fa_bwd_workspace_size(a["B"], a["Sq"], a["H"])
+    return lib.fa_bwd(a["dout"], a["q"], a["k"], a["v"], a["out"], a["lse"], a["dq"], a["dk"],
+                      a["dv"], a["dtype"], a["B"], a["Sq"], a["Sk"], a["H"], a["Hkv"], a["d"],
+                      a["scale"], a["causal"], a["wl"], a["wr"], a["softcap"], a["alibi"],
+                      a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), FA_ERR_UNSUPPORTED),
+    (dict(dtype=2), FA_ERR_UNSUPPORTED),
+    (dict(softcap=30.0), FA_ERR_UNSUPPORTED),               # no softcap in the backward
+    (dict(H=3, Hkv=2), FA_ERR_INVALID_ARG),
+    (dict(dout=None), FA_ERR_INVALID_ARG),
+    (dict(lse=None), FA_ERR_INVALID_ARG),
+    (dict(dk=MIS), FA_ERR_INVALID_ARG),
+    (dict(lse=ctypes.c_void_p(0x10002)), FA_ERR_INVALID_ARG),  # lse must be 4-byte aligned
+    (dict(Sk=-1), FA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), FA_ERR_INVALID_ARG),
+    (dict(ws=None), FA_ERR_WORKSPACE),
+    (dict(ws_bytes=16), FA_ERR_WORKSPACE),
+    (dict(ws=MIS), FA_ERR_WORKSPACE),
+])
+def test_bwd_validation(lib, kw, code):
+    assert bwd(lib, **kw) == code
+    assert lib.fa_last_error()
+
+
+def test_bwd_workspace_size(lib):
+    # two fp32 arrays (D and LSE * log2 e), rows padded to a multiple of 4, the total
+    # rounded up to 256 bytes
+    def up256(n):
+        return (n + 255) // 256 * 256
+    assert lib.fa_bwd_workspace_size(2, 130, 3) == up256(2 * 2 * 3 * 132 * 4)
+    assert lib.fa_bwd_workspace_size(1, 128, 1) == up256(2 * 128 * 4)
+    assert lib.fa_bwd_workspace_size(0, 128, 1) == 256
+
+
+def test_bwd_empty_batch_is_a_noop(lib):
+    assert bwd(lib, B=0) == FA_OK
