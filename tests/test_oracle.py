@@ -447,3 +447,68 @@ def test_append_then_attend_equals_attention_on_the_concatenation():
         o1, l1 = oracle.attention_dense(q[b:b + 1], kc, vc, causal=True)
         np.testing.assert_allclose(out[b], o1[0], rtol=0, atol=1e-12)
         np.testing.assert_allclose(lse[b], l1[0], rtol=0, atol=1e-12)
+
+
+def brute_attention(q, k, v, scale, causal, window, softcap, slopes):
+    """Per-element pure-Python fp64 attention (math.exp / math.tanh), written out
+    from the definition: bottom-right aligned mask, softcap inside the exponent,
+    ALiBi as -slope * |i + Sk - Sq - j|, empty rows give O = 0 and LSE = -inf."""
+    B, Sq, H, d = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = H // Hkv
+    wl, wr = window
+    out = np.zeros((B, Sq, H, d))
+    lse = np.full((B, H, Sq), -math.inf)
+    for b in range(B):
+        for h in range(H):
+            hk = h // G
+            for i in range(Sq):
+                c = i + Sk - Sq
+                scores = []
+                for j in range(Sk):
+                    if causal and j > c:
+                        continue
+                    if wl >= 0 and j < c - wl:
+                        continue
+                    if not causal and wr >= 0 and j > c + wr:
+                        continue
+                    s = scale * sum(float(q[b, i, h, t]) * float(k[b, j, hk, t]) for t in range(d))
+                    if softcap > 0:
+                        s = softcap * math.tanh(s / softcap)
+                    if slopes is not None:
+                        s -= float(slopes[h]) * abs(c - j)
+                    scores.append((j, s))
+                if not scores:
+                    continue
+                m = max(s for _, s in scores)
+                z = sum(math.exp(s - m) for _, s in scores)
+                lse[b, h, i] = m + math.log(z)
+                for j, s in scores:
+                    w = math.exp(s - lse[b, h, i])
+                    for t in range(d):
+                        out[b, i, h, t] += w * float(v[b, j, hk, t])
+    return out, lse
+
+
+@pytest.mark.parametrize("sq,sk", [(4, 4), (3, 7), (6, 2)])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("window", [(-1, -1), (1, -1), (-1, 1), (2, 0)])
+@pytest.mark.parametrize("softcap", [0.0, 1.5])
+@pytest.mark.parametrize("alibi", [False, True])
+def test_brute_force_every_flag_combination(sq, sk, causal, window, softcap, alibi):
+    """Tiny shapes (B=2, H=2 over Hkv=1, d=3), every flag combination, against the
+    per-element pure-Python definition above: agreement to 1e-12."""
+    rng = np.random.default_rng(sq * 100 + sk * 10 + causal)
+    q = rng.standard_normal((2, sq, 2, 3))
+    k = rng.standard_normal((2, sk, 1, 3))
+    v = rng.standard_normal((2, sk, 1, 3))
+    slopes = np.array([0.5, 0.125]) if alibi else None
+    kw = dict(scale=0.8, causal=causal, window=window, softcap=softcap)
+    if alibi:
+        kw["alibi_slopes"] = slopes
+    o, l = oracle.attention_dense(q, k, v, **kw)
+    ro, rl = brute_attention(q, k, v, 0.8, causal, window, softcap, slopes)
+    np.testing.assert_allclose(o, ro, atol=1e-12, rtol=0)
+    assert np.array_equal(np.isneginf(l), np.isneginf(rl))
+    fin = np.isfinite(rl)
+    np.testing.assert_allclose(l[fin], rl[fin], atol=1e-12, rtol=0)
