@@ -21,9 +21,11 @@
 // Roles per CTA (384 threads): warps 0-7 compute in two warpgroups that split
 // each block's columns (thread r of a warpgroup owns tensor-memory lane r: a key
 // row in dK/dV, a query row in dQ), warp 8 TMA producer, warp 9 MMA issuer (one
-// elected thread; it also allocates tensor memory), warps 10-11 idle.  Tensor memory: S [0,128), dP [128,256), accumulators from 256; P and dS
-// are written as 16-bit pairs over the first 64 columns of S and dP, which the
-// thread has already read.  Every wait is bounded.
+// elected thread; it also allocates tensor memory), warps 10-11 idle.  Tensor
+// memory of the dK/dV kernel: S^T [0,128), dP^T [128,256), dV and dK from 256; P^T
+// and dS^T are written as 16-bit pairs over the first 64 columns of S^T and dP^T
+// once those scores are in registers (warpgroup 1 waits for warpgroup 0's read).
+// The dQ kernel's layout is given above it.  Every wait is bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -139,8 +141,9 @@ __global__ void __launch_bounds__(256) bwd_dot_kernel(const BwdParams p) {
   const bool live = row < static_cast<int64_t>(p.B) * p.Sq * p.H;
   float acc = 0.f;
   if (live) {
-    const uint4 o = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.out) + row * D + l * 8);
-    const uint4 g = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + row * D + l * 8);
+    const int64_t at = row * D + l * 8;
+    const uint4 o = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.out) + at);
+    const uint4 g = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + at);
     const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
