@@ -110,7 +110,13 @@ def _check(rc: int):
 
 
 def _ptr(t) -> ctypes.c_void_p | None:
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a CUDA tensor (None stays NULL).  Host tensors, pinned ones
+    included, are refused: every pointer of the C ABI is read by the kernels."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"tensor arguments must be CUDA tensors, got one on {t.device}")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _i64(vals) -> ctypes.Array:

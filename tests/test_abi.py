@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import io_aware_online_b200 as fa
 from io_aware_online_b200 import build as fa_build
@@ -236,3 +237,14 @@ def test_bwd_workspace_size(lib):
 
 def test_bwd_empty_batch_is_a_noop(lib):
     assert bwd(lib, B=0) == FA_OK
+
+
+def test_binding_refuses_host_tensors(lib):
+    """The binding passes device addresses only: a host tensor is refused before
+    any call into the library (stream=0 keeps the call free of CUDA on this host)."""
+    q = torch.zeros(1, 128, 2, 64, dtype=torch.float16)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        fa.fa_fwd(q, q, q, stream=0)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        fa.fa_bwd(q, q, q, q, q, torch.zeros(1, 2, 128), dq=q, dk=q, dv=q,
+                  workspace=torch.zeros(4096, dtype=torch.uint8), stream=0)
