@@ -135,10 +135,11 @@ FA_API int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out, fl
 
 /*
  * fa_kvcache_num_splits -- the split count fa_fwd_kvcache uses for these sizes.
- * num_splits > 0 is returned unchanged (clamped to the number of cache pages);
- * 0 asks for the library's heuristic, which depends only on the arguments and on
- * the current device's SM count.  max_seqlen_k is the largest cache length
- * (max_blocks_per_seq * page_size for a paged cache).  Returns <= 0 on bad input.
+ * num_splits in 1..256 is returned unchanged apart from a clamp to the number of
+ * cache pages; 0 asks for the library's heuristic, which depends only on the
+ * arguments and on the current device's SM count.  max_seqlen_k is the largest
+ * cache length (max_blocks_per_seq * page_size for a paged cache).  Returns <= 0
+ * on bad input, including num_splits < 0 or > 256.
  */
 FA_API int fa_kvcache_num_splits(int batch, int seqlen_q, int num_heads, int num_heads_k,
                           int head_dim, int max_seqlen_k, int page_size, int num_splits);
@@ -172,7 +173,8 @@ FA_API size_t fa_kvcache_workspace_size(int batch, int seqlen_q, int num_heads, 
  * cache_seqlens: int32 [batch], the number of keys sequence b attends (its query
  *   rows sit at key positions cache_seqlens[b] - seqlen_q ..).  NULL means
  *   seqlen_k_max for every sequence (contiguous cache only).
- * num_splits: 0 = heuristic; otherwise the keys of each sequence are cut, at
+ * num_splits: 0 = heuristic; 1..256 (larger counts return FA_ERR_INVALID_ARG:
+ *   the combine step weighs at most 256 partials); otherwise the keys of each sequence are cut, at
  *   page granularity (64-token chunks for a contiguous cache), into num_splits
  *   ranges of ceil(pages / num_splits) pages, each computed by its own CTAs, and a
  *   second kernel combines them (fa_combine's arithmetic).  The result does not
@@ -297,16 +299,19 @@ FA_API int fa_selftest_wait_timeout(int timeout_ms, void *stream);
  * that owns every device allocation through its own pool, or a serving loop that
  * must not risk the device synchronisation a cudaMalloc can cause).  The pages
  * have no counterpart to this call.  It allocates nothing: its scratch (the
- * work-item counter and the fp32 split partials) is one fixed 16 MiB array in
+ * work-item counter and the fp32 split partials) is one fixed 24 MiB array in
  * device memory (fa_kvcache_static_scratch_bytes()), present on every GPU that
- * loads the library until the process exits.  Arguments and results are those of
+ * loads the library until the process exits; it holds, for example, the partials
+ * of a 64-sequence, 32-head, head-dim-128 single-token decode at up to 23 splits.  Arguments and results are those of
  * fa_fwd_kvcache.  A call whose need (fa_kvcache_workspace_size) exceeds the array
  * returns FA_ERR_WORKSPACE without launching anything.  All calls share the array
  * and it keeps the last call's contents; each call clears the counter on its own
  * stream, so calls that overlap on the GPU race and must be serialised by the
  * caller.  The first call on a device looks the array's address up
  * (cudaGetSymbolAddress) with that device current; make it before any stream
- * capture.
+ * capture.  The address stays cached for the life of the process, so after a
+ * device reset (cudaDeviceReset, or the primary context released and created
+ * again) this call must not be used any more.
  */
 FA_API int fa_fwd_kvcache_static(const void *q, const void *k_cache, const void *v_cache,
                                  void *out, float *lse, int dtype, int batch, int seqlen_q,

@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -162,10 +163,16 @@ void fill_score_params(float scale, float softcap, float* scale_log2, float* sof
   *tanh_k = softcap > 0.f ? 2.f * log2e * scale / softcap : 0.f;
 }
 
+// Largest split count: the combine kernel keeps one weight per split in shared
+// memory (kCombineMaxSplits in combine.cu).
+constexpr int kMaxSplits = 256;
+
 int resolve_splits(int batch, int Sq, int H, int Hkv, int d, int max_seqlen_k, int unit,
                    int num_splits) {
   (void)Sq; (void)H; (void)d;
-  if (batch < 0 || Hkv <= 0 || max_seqlen_k < 0 || unit <= 0 || num_splits < 0) return -1;
+  if (batch < 0 || Hkv <= 0 || max_seqlen_k < 0 || unit <= 0 || num_splits < 0 ||
+      num_splits > kMaxSplits)
+    return -1;
   const int units = std::max(1, (max_seqlen_k + unit - 1) / unit);
   if (num_splits > 0) return std::min(num_splits, units);
   // heuristic: about eight work items per resident decode CTA (three per SM), so the
@@ -366,6 +373,7 @@ static bool kvcache_uses_prefill(int seqlen_q, int num_heads, int num_heads_k) {
 
 int fa_kvcache_num_splits(int batch, int seqlen_q, int num_heads, int num_heads_k, int head_dim,
                           int max_seqlen_k, int page_size, int num_splits) {
+  if (num_splits < 0 || num_splits > kMaxSplits) return -1;
   if (kvcache_uses_prefill(seqlen_q, num_heads, num_heads_k)) return 1;  // no split partials
   const int unit = page_size > 0 ? page_size : 64;
   return resolve_splits(batch, seqlen_q, num_heads, num_heads_k, head_dim, max_seqlen_k, unit,
@@ -405,6 +413,8 @@ static int kvcache_impl(const void* q, const void* k_cache, const void* v_cache,
     return fail(FA_ERR_INVALID_ARG, "fa_fwd_kvcache: q, caches and out must be 16-byte aligned");
   if (batch < 0 || seqlen_q < 0 || num_splits < 0)
     return fail(FA_ERR_INVALID_ARG, "fa_fwd_kvcache: negative size");
+  if (num_splits > kMaxSplits)
+    return fail(FA_ERR_INVALID_ARG, "fa_fwd_kvcache: num_splits must be in [0, %d]", kMaxSplits);
   const int H = num_heads, Hkv = num_heads_k, d = head_dim, G = H / Hkv;
   const bool use_prefill = kvcache_uses_prefill(seqlen_q, H, Hkv);
   const bool paged = block_table != nullptr;
@@ -416,6 +426,8 @@ static int kvcache_impl(const void* q, const void* k_cache, const void* v_cache,
       return fail(FA_ERR_INVALID_ARG, "fa_fwd_kvcache: num_blocks and max_blocks_per_seq must be positive");
     if (cache_seqlens == nullptr)
       return fail(FA_ERR_INVALID_ARG, "fa_fwd_kvcache: a paged cache needs cache_seqlens");
+    if (static_cast<int64_t>(max_blocks_per_seq) * page_size > INT_MAX)
+      return fail(FA_ERR_INVALID_ARG, "fa_fwd_kvcache: max_blocks_per_seq * page_size overflows int");
     max_k = max_blocks_per_seq * page_size;
     unit = page_size;
   } else {

@@ -11,8 +11,9 @@
 // no cudaMalloc, no cudaFree, no allocating library routine.
 //
 // Costs and rules of the fixed array:
-// - it is kFaStaticScratchBytes (16 MiB) on every GPU where the library is
-//   loaded, held until the process exits;
+// - it is kFaStaticScratchBytes (24 MiB) on every GPU where the library is
+//   loaded, held until the process exits.  That holds the split partials of a
+//   64-sequence, 32-head, head-dim-128 decode at up to 23 splits;
 // - a call whose scratch need (fa_kvcache_workspace_size) exceeds it is
 //   rejected with FA_ERR_WORKSPACE before anything is launched;
 // - all calls share the array and it keeps the last call's contents; what must
@@ -21,17 +22,20 @@
 //   serialised by the caller;
 // - the first call on each device looks the array's device address up with
 //   cudaGetSymbolAddress, with that device current; make that first call before
-//   any stream capture.
+//   any stream capture.  The address is cached for the life of the process: after
+//   a device reset (cudaDeviceReset, or the primary context released and made
+//   again) the cached address is stale and this entry point must not be called.
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cstdio>
 #include <mutex>
 
 #include "fa.h"
 #include "fa_internal.h"
 
-// 16 MiB, 256-byte aligned: the fixed scratch of fa_fwd_kvcache_static.
-static constexpr size_t kFaStaticScratchBytes = size_t(16) << 20;
+// 24 MiB, 256-byte aligned: the fixed scratch of fa_fwd_kvcache_static.
+static constexpr size_t kFaStaticScratchBytes = size_t(24) << 20;
 static __device__ __align__(256) unsigned char g_fa_static_scratch[kFaStaticScratchBytes];
 
 namespace {
@@ -72,7 +76,14 @@ FA_API int fa_fwd_kvcache_static(const void* q, const void* k_cache, const void*
                                  int window_left, int window_right, float softcap,
                                  const float* alibi_slopes, int num_splits, void* stream) {
   const bool paged = block_table != nullptr;
-  const int max_k = paged ? max_blocks_per_seq * page_size : seqlen_k_max;
+  // the arguments the size check reads are validated first, so that a malformed call
+  // gets the same FA_ERR_INVALID_ARG as from fa_fwd_kvcache, not a scratch-size error
+  const int64_t max_k64 = paged ? static_cast<int64_t>(max_blocks_per_seq) * page_size
+                                : static_cast<int64_t>(seqlen_k_max);
+  if (max_k64 < 0 || max_k64 > INT_MAX || num_splits < 0 || num_splits > 256)
+    return fa::set_error(FA_ERR_INVALID_ARG,
+                         "fa_fwd_kvcache_static: cache extent or num_splits out of range");
+  const int max_k = static_cast<int>(max_k64);
   const size_t need = fa_kvcache_workspace_size(batch, seqlen_q, num_heads, num_heads_k,
                                                 head_dim, max_k, paged ? page_size : 0,
                                                 num_splits);

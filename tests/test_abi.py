@@ -110,6 +110,12 @@ def kvc(lib, **kw):
     (dict(splits=4, ws=None, wsb=0), FA_ERR_WORKSPACE),
     (dict(splits=1, ws=None, wsb=0), FA_ERR_WORKSPACE),       # the item counter lives there
     (dict(bt=None, skmax=-1), FA_ERR_INVALID_ARG),
+    # the combine step weighs at most 256 partials: larger split counts are refused
+    # before any device use (also on the path whose need fits a workspace)
+    (dict(splits=257, ws=P, wsb=1 << 40), FA_ERR_INVALID_ARG),
+    (dict(splits=512, maxb=1024, ws=P, wsb=1 << 40), FA_ERR_INVALID_ARG),
+    # max_blocks_per_seq * page_size must fit an int
+    (dict(maxb=1 << 24, page=256, ws=P, wsb=1 << 40), FA_ERR_INVALID_ARG),
 ])
 def test_kvcache_validation(lib, kw, code):
     assert kvc(lib, **kw) == code
@@ -124,6 +130,26 @@ def test_splits_and_workspace_size(lib):
     # more than 16 query rows per KV head run the tensor-core kernel: no split partials
     assert lib.fa_kvcache_num_splits(4, 128, 32, 8, 128, 32768, 256, 16) == 1
     assert lib.fa_kvcache_workspace_size(4, 128, 32, 8, 128, 32768, 256, 16) == 256
+    # split counts above 256 (the combine's limit) are bad input, whatever the route
+    assert lib.fa_kvcache_num_splits(1, 1, 8, 8, 128, 1 << 20, 256, 256) == 256
+    assert lib.fa_kvcache_num_splits(1, 1, 8, 8, 128, 1 << 20, 256, 257) <= 0
+    assert lib.fa_kvcache_num_splits(4, 128, 32, 8, 128, 32768, 256, 300) <= 0
+    assert lib.fa_kvcache_workspace_size(1, 1, 8, 8, 128, 1 << 20, 256, 512) == 256
+
+
+def test_static_scratch_validation(lib):
+    # the arguments the scratch-size check reads are validated first: a malformed
+    # call gets FA_ERR_INVALID_ARG, as from fa_fwd_kvcache, before any device use
+    st = lib.fa_fwd_kvcache_static
+    args = [P, P, P, P, None, 1, 64, 1, 32, 8, 128, P, 128, 256, 8192, 0, P, float("nan"), 1,
+            -1, -1, 0.0, None]
+    assert st(*args, 300, None) == FA_ERR_INVALID_ARG             # num_splits > 256
+    big = list(args)
+    big[12] = 1 << 24                                             # max_blocks_per_seq * page
+    assert st(*big, 4, None) == FA_ERR_INVALID_ARG
+    # 64 x 32 x 129 fp32 partials at 128 splits need ~135 MB: beyond the fixed array
+    assert st(*args, 128, None) == FA_ERR_WORKSPACE
+    assert lib.fa_kvcache_static_scratch_bytes() == 24 << 20
 
 
 def test_combine_validation(lib):

@@ -6,14 +6,16 @@ It runs the same split-KV decode with its scratch in the library's fixed device
 array.  Checked through the C ABI against fa_fwd_kvcache (caller workspace) on the
 same inputs, within the decode tolerances, on two calls in a row: the array keeps
 the previous call's contents, so the second call also shows that what must start
-at zero is cleared.  The file sorts last so that a run stopping at the first
-failure has already run every other test.
+at zero is cleared.  Each call is also checked against the fp64 oracle directly.
+The file sorts last so that a run stopping at the first failure has already run
+every other test.
 """
 import ctypes
 
 import pytest
 import torch
 
+import oracle
 import synth
 from parity import check_lse, check_out, to_np
 
@@ -26,11 +28,12 @@ def test_static_scratch_decode_matches_workspace_decode():
     from io_aware_online_b200 import build
     build.build()
     lib = fa.load()
-    assert lib.fa_kvcache_static_scratch_bytes() == 16 << 20
+    assert lib.fa_kvcache_static_scratch_bytes() == 24 << 20
     lens = [1, 300, 2048, 4097, 777, 64]
     H, Hkv, d, page = 32, 8, 128, 256
     kp, vp, bt, cs = synth.paged_cache(lens, page, Hkv, d, torch.bfloat16, seed=91, spare_blocks=2)
     q = synth.randn((len(lens), 1, H, d), torch.bfloat16, torch.Generator().manual_seed(92))
+    ro, rl = oracle.attention_paged(q, kp, vp, bt, cs, causal=True)
     kp, vp, bt, cs, q = kp.to(DEV), vp.to(DEV), bt.to(DEV), cs.to(DEV), q.to(DEV)
     for splits in (4, 16):
         ref_o, ref_l = fa.fa_fwd_kvcache(q, kp, vp, cache_seqlens=cs, block_table=bt,
@@ -49,13 +52,15 @@ def test_static_scratch_decode_matches_workspace_decode():
             torch.cuda.synchronize()
             check_out(out, to_np(ref_o), torch.bfloat16, what=f"O (splits {splits}, call {call})")
             check_lse(lse, to_np(ref_l), what=f"LSE (splits {splits}, call {call})")
+            check_out(out, ro, torch.bfloat16, what=f"O vs oracle (splits {splits}, call {call})")
+            check_lse(lse, rl, what=f"LSE vs oracle (splits {splits}, call {call})")
     assert fa.fa_device_status(clear=True) == 0
 
 
 def test_static_scratch_rejects_oversized_calls():
     import io_aware_online_b200 as fa
     lib = fa.load()
-    # 64 sequences x 32 heads x 129 floats x 256 splits is far beyond 16 MiB
+    # 64 sequences x 32 heads x 129 floats x 128 splits (~135 MB) is far beyond 24 MiB
     q = torch.zeros(64, 1, 32, 128, dtype=torch.bfloat16, device=DEV)
     kp = torch.zeros(300, 256, 8, 128, dtype=torch.bfloat16, device=DEV)
     bt = torch.zeros(64, 128, dtype=torch.int32, device=DEV)
