@@ -95,6 +95,11 @@ enum fa_device_flag {
  *   contiguous layout above.  In varlen mode entry 0 is ignored.  Every stride must
  *   be a multiple of 8 elements (16 bytes) and every pointer 16-byte aligned.
  * lse may be NULL.  The N x N score matrix is never written to memory.
+ * Errors: argument errors return FA_ERR_* before anything is launched.  A
+ * pipeline wait inside the kernel that runs past its limit (fa_set_wait_timeout_ms)
+ * stops that CTA and raises FA_DEV_WAIT_TIMEOUT in the device status word
+ * (fa_device_status); out and lse of a call after which that bit is set are
+ * undefined: the stopped CTA's rows may hold partial results or stale memory.
  */
 FA_API int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int dtype,
            int batch, int seqlen_q, int seqlen_k, int num_heads, int num_heads_k, int head_dim,

@@ -272,7 +272,8 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* out, floa
     return fail(FA_ERR_UNSUPPORTED, "fa_fwd: batch (%d) or query tiles (%d) above 65535", batch, n_tiles);
   if ((rc = get_encoder()) != FA_OK) return rc;
   unsigned int* status = nullptr;
-  if ((rc = device_state(nullptr, &status, nullptr)) != FA_OK) return rc;
+  int sms = 0;
+  if ((rc = device_state(nullptr, &status, &sms)) != FA_OK) return rc;
 
   CUtensorMap tq, tk, tv;
   // one 128-byte swizzle atom per row of the box: 64 16-bit or 128 8-bit elements
@@ -322,6 +323,12 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* out, floa
   p.wl = window_left;
   p.wr = window_right;
   p.tile_major = (!causal && window_left < 0 && window_right < 0) ? 1 : 0;
+  // dense calls run a persistent grid; under a mask the work of a unit grows with
+  // its row index, and pairing the heaviest unit with the lightest evens it out
+  p.persistent = varlen ? 0 : 1;
+  p.pair = (causal || window_left >= 0 || window_right >= 0) ? 1 : 0;
+  p.B = batch;
+  p.sm_count = sms;
   p.status = status;
   p.timeout_ns = timeout_ns();
   cudaStream_t st = static_cast<cudaStream_t>(stream);

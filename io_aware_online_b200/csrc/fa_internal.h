@@ -24,6 +24,10 @@ struct FwdParams {
   const float* alibi;              // [H] or NULL
   int causal, wl, wr;              // mask flags; -1 = unbounded window side
   int tile_major;                  // grid x = query tiles (no mask: equal work per tile)
+  // persistent schedule (dense calls): CTA c takes items c, c + gridDim.x, ... of the
+  // (batch, head, pair) order; pair: an item is units n-1-u and u of one head
+  int persistent, pair, B;
+  int sm_count;                    // SMs of the device (persistent grid size)
   float v_descale;                 // 8-bit inputs: O is multiplied by it (1 otherwise)
   // KV-cache mode (fa_fwd_kvcache with many query rows): K/V come from a paged pool
   // [num_blocks, page, Hkv, D] through block_table, or from a contiguous cache

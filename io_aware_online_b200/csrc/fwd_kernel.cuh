@@ -30,7 +30,20 @@
 // The running max is kept lazily: O is rescaled only when a row's max grows by
 // more than 8 (base-2 units); the final O / l and LSE use the same stale max, so
 // the result is unchanged.  Blocks that lie fully inside every row's allowed key
-// range skip the mask; blocks outside the CTA's key range are never loaded.
+// range skip the mask; blocks outside the unit's key range are never loaded.
+//
+// Work schedule.  A "unit" is the T query tiles (T * 128 rows) of one (sequence,
+// head).  Dense calls run persistently: the grid holds as many CTAs as fit on the
+// device at once and CTA c takes work items c, c + gridDim.x, ...; items are
+// ordered (batch, head)-major so that the CTAs running at any moment share a few
+// heads' K/V in L2.  Under a causal or window mask an item pairs unit n-1-u with
+// unit u of the same head (the heaviest with the lightest), so every item carries
+// the same number of key blocks and a static assignment stays balanced.  The
+// roles of a CTA walk the same unit sequence; ring slots and barrier phases run on
+// across units, and the next unit's Q is loaded as soon as the last product that
+// reads the current Q has completed, so one unit's epilogue overlaps the next
+// unit's first products.  Varlen and KV-cache calls take one unit per CTA, the
+// heaviest units first.
 #pragma once
 
 #include <climits>
@@ -65,7 +78,7 @@ struct FwdCfg {
   static constexpr int kThreads = (4 * T + 4) * 32;   // softmax warpgroups + one more
   static constexpr int kMinBlocks = 3 - T;             // CTAs per SM
   // registers a thread launches with, and what the non-softmax warpgroup keeps:
-  // T*128*200 + 128*kOtherRegs = kThreads * kLaunchRegs
+  // T*128*kSoftmaxRegs + 128*kOtherRegs = kThreads * kLaunchRegs
   static constexpr int kLaunchRegs = (T == 2) ? 168 : 128;
   static constexpr uint32_t kOtherRegs = (T == 2) ? 104 : 56;
   static_assert(T * 128 * kSoftmaxRegs + 128 * kOtherRegs == kThreads * kLaunchRegs,
@@ -80,8 +93,8 @@ struct FwdCfg {
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
-  // o_final[2], drain[2], s_free[2], pv_done[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 12;
+  // o_final[2], drain[2], s_free[2], pv_done[2], q_empty
+  static constexpr int kNumBars = 1 + 4 * kStages + 13;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // room to align the base to 1 KiB
@@ -107,6 +120,87 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint6
   return true;
 }
 
+// One unit of work: query rows [row0, row0 + T*128) of sequence b, head h, and the
+// key blocks [j_lo, j_lo + n_blk) they may attend.
+struct FwdUnit {
+  int state;               // 0: no more units; 1: nothing at this position; 2: a unit
+  int b, h;
+  int q0, k0, Sq_b, Sk_b;  // varlen row offsets and this sequence's lengths
+  int row0, off;           // first query row; key offset of the bottom-right alignment
+  int j_lo, n_blk;
+};
+
+// The k-th unit of this CTA (state 0 = no more units, 1 = none at this position,
+// 2 = a unit).  Persistent schedule (dense): item = blockIdx.x + m * gridDim.x,
+// items ordered (batch, head, pair index); with pairing, k = 2m takes unit
+// n-1-pi and k = 2m+1 unit pi of pair pi.  Otherwise one unit per CTA from
+// blockIdx, heaviest first.
+template <int T, bool KV>
+__device__ __forceinline__ FwdUnit fwd_unit_at(const FwdParams& p, int k) {
+  FwdUnit u{};
+  int b, h, unit;
+  int q0 = 0, k0 = 0, Sq_b = p.Sq, Sk_b = p.Sk;
+  if (p.persistent) {
+    const int n_units = (p.Sq + T * kBM - 1) / (T * kBM);
+    const int n_pi = p.pair ? (n_units + 1) / 2 : n_units;
+    const int per = p.pair ? 2 : 1;
+    const int item = blockIdx.x + (k / per) * gridDim.x;
+    if (item >= p.B * p.H * n_pi) return u;  // state 0
+    const int pi = item % n_pi;
+    const int bh = item / n_pi;
+    b = bh / p.H;
+    h = bh % p.H;
+    if (p.pair) {
+      unit = (k % 2 == 0) ? n_units - 1 - pi : pi;
+      if (k % 2 == 1 && unit == n_units - 1 - pi) {  // middle unit of an odd count
+        u.state = 1;
+        return u;
+      }
+    } else {
+      unit = pi;
+    }
+  } else {
+    if (k > 0) return u;
+    h = p.tile_major ? blockIdx.y : blockIdx.x;
+    b = p.tile_major ? blockIdx.z : blockIdx.y;
+    const int zi = static_cast<int>(p.tile_major ? blockIdx.x : blockIdx.z);
+    if (p.cu_q != nullptr) {
+      q0 = p.cu_q[b];
+      Sq_b = p.cu_q[b + 1] - q0;
+      k0 = p.cu_k[b];
+      Sk_b = p.cu_k[b + 1] - k0;
+    } else if (KV) {
+      Sk_b = ((p.cache_seqlens != nullptr) ? p.cache_seqlens[b] : p.Sk) + p.k_add;
+      // a length the cache cannot hold would read past the block table: clamp, report
+      const int cap = (p.block_table != nullptr) ? p.max_blocks * p.page_size : p.Sk;
+      if (Sk_b < 0 || Sk_b > cap) {
+        if (threadIdx.x == 0) atomicOr(p.status, kDevBadLength);
+        Sk_b = min(max(Sk_b, 0), cap);
+      }
+    }
+    const int n_units_b = (Sq_b + T * kBM - 1) / (T * kBM);
+    if (zi >= n_units_b) return u;
+    unit = n_units_b - 1 - zi;  // heaviest rows first
+  }
+  u.b = b;
+  u.h = h;
+  u.q0 = q0;
+  u.k0 = k0;
+  u.Sq_b = Sq_b;
+  u.Sk_b = Sk_b;
+  u.row0 = unit * T * kBM;
+  u.off = Sk_b - Sq_b;
+  // the unit's key range: [lo(first row), hi(last row)] intersected with [0, Sk_b)
+  const int right = p.causal ? 0 : p.wr;
+  const int r_last = min(u.row0 + T * kBM - 1, Sq_b - 1);
+  const int k_begin = (p.wl >= 0) ? max(0, u.row0 + u.off - p.wl) : 0;
+  const int k_end = ((p.causal || p.wr >= 0) ? min(r_last + u.off + right, Sk_b - 1) : Sk_b - 1) + 1;
+  u.j_lo = k_begin / kBN;
+  u.n_blk = (k_end > k_begin) ? (k_end + kBN - 1) / kBN - u.j_lo : 0;
+  u.state = 2;
+  return u;
+}
+
 // EMU: of every 8 pairs of probabilities, EMU are evaluated by exp2_fma2 on the
 // FMA pipe and the rest by the MUFU unit (balances the two at small head dims).
 // S_t = Q_t K^T into tensor memory: K-major A (Q tile) and B (K block); a step of
@@ -114,34 +208,53 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint6
 // lies 16 KiB further.
 // With 8-bit inputs (E = 1) a step is 32 elements, still 32 bytes, through
 // tcgen05.mma kind::f8f6f4.
+// Descriptors are passed as their low words (start address, leading offset) plus
+// the high word they share (stride offset, version, swizzle mode); a step adds
+// its byte offset / 16 to the start address field, which cannot carry.
+template <int D, int E = 2>
+__device__ __forceinline__ void fwd_issue_qk(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                             uint32_t hi, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < D * E / 32; ++kk) {
+    const uint32_t o = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+    if constexpr (E == 2)
+      mma_ss(d_tmem, desc_pack(a_lo + o, hi), desc_pack(b_lo + o, hi), idesc, kk > 0 ? 1u : 0u);
+    else
+      mma_ss_f8(d_tmem, desc_pack(a_lo + o, hi), desc_pack(b_lo + o, hi), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// The same product from two full descriptors (their high words must agree: every
+// 128-byte-swizzled operand here has a 1 KiB stride offset).
 template <int D, int E = 2>
 __device__ __forceinline__ void fwd_issue_qk(uint32_t d_tmem, uint64_t a0, uint64_t b0,
                                              uint32_t idesc) {
-#pragma unroll
-  for (int kk = 0; kk < D * E / 32; ++kk) {
-    const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
-    if constexpr (E == 2)
-      mma_ss(d_tmem, desc_advance(a0, o), desc_advance(b0, o), idesc, kk > 0 ? 1u : 0u);
-    else
-      mma_ss_f8(d_tmem, desc_advance(a0, o), desc_advance(b0, o), idesc, kk > 0 ? 1u : 0u);
-  }
+  fwd_issue_qk<D, E>(d_tmem, static_cast<uint32_t>(a0), static_cast<uint32_t>(b0),
+                     static_cast<uint32_t>(a0 >> 32), idesc);
 }
 
 // O_t (+)= P_t V: A = P from tensor memory (8 columns hold 16 keys), B = V block,
 // MN-major (16 keys = 16 rows = 2 KiB; head-dim atoms 16 KiB apart).
 // With 8-bit P and V a step is 32 keys: 8 columns of four E4M3 values, 4 KiB of V.
 template <int D, int E = 2>
-__device__ __forceinline__ void fwd_issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
-                                             uint32_t idesc, bool acc) {
+__device__ __forceinline__ void fwd_issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                             uint32_t b_hi, uint32_t idesc, bool acc) {
 #pragma unroll
   for (int kk = 0; kk < kBN * E / 32; ++kk) {
     if constexpr (E == 2)
-      mma_ts(d_tmem, a_tmem + kk * 8, desc_advance(b0, kk * 2048), idesc,
+      mma_ts(d_tmem, a_tmem + kk * 8, desc_pack(b_lo + kk * (2048 >> 4), b_hi), idesc,
              (acc || kk > 0) ? 1u : 0u);
     else
-      mma_ts_f8(d_tmem, a_tmem + kk * 8, desc_advance(b0, kk * 4096), idesc,
+      mma_ts_f8(d_tmem, a_tmem + kk * 8, desc_pack(b_lo + kk * (4096 >> 4), b_hi), idesc,
                 (acc || kk > 0) ? 1u : 0u);
   }
+}
+
+template <int D, int E = 2>
+__device__ __forceinline__ void fwd_issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
+                                             uint32_t idesc, bool acc) {
+  fwd_issue_pv<D, E>(d_tmem, a_tmem, static_cast<uint32_t>(b0), static_cast<uint32_t>(b0 >> 32),
+                     idesc, acc);
 }
 
 // FP8: E4M3 Q, K, V (both products on kind::f8f6f4, P rounded to E4M3), bf16 output
@@ -163,46 +276,6 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  // grid order: query tiles fastest when every tile does the same work (the
-  // tiles of a head then run together and share its K/V in L2), else heads
-  // fastest with the heaviest tiles first (balance under a causal or window mask)
-  const int h = p.tile_major ? blockIdx.y : blockIdx.x;
-  const int b = p.tile_major ? blockIdx.z : blockIdx.y;
-  const int zi = static_cast<int>(p.tile_major ? blockIdx.x : blockIdx.z);
-  const int hk = h / p.G;
-
-  // ---------------------------------------------------------- problem geometry
-  int q0 = 0, k0 = 0, Sq_b = p.Sq, Sk_b = p.Sk;
-  if (p.cu_q != nullptr) {
-    q0 = p.cu_q[b];
-    Sq_b = p.cu_q[b + 1] - q0;
-    k0 = p.cu_k[b];
-    Sk_b = p.cu_k[b + 1] - k0;
-  } else if (KV) {
-    Sk_b = ((p.cache_seqlens != nullptr) ? p.cache_seqlens[b] : p.Sk) + p.k_add;
-    // a length the cache cannot hold would read past the block table: clamp, report
-    const int cap = (p.block_table != nullptr) ? p.max_blocks * p.page_size : p.Sk;
-    if (Sk_b < 0 || Sk_b > cap) {
-      if (threadIdx.x == 0) atomicOr(p.status, kDevBadLength);
-      Sk_b = min(max(Sk_b, 0), cap);
-    }
-  }
-  const int n_units_b = (Sq_b + T * kBM - 1) / (T * kBM);
-  if (zi >= n_units_b) return;  // uniform: whole CTA leaves
-  const int unit = n_units_b - 1 - zi;  // heaviest rows first
-  const int row0 = unit * T * kBM;
-  const int off = Sk_b - Sq_b;  // bottom-right alignment
-  const bool has_left = p.wl >= 0;
-  const bool has_right = p.causal || p.wr >= 0;
-  const int right = p.causal ? 0 : p.wr;
-  // allowed keys of row i: [lo(i), hi(i)] intersected with [0, Sk_b)
-  auto lo_of = [&](int i) { return has_left ? i + off - p.wl : INT_MIN / 2; };
-  auto hi_of = [&](int i) { return has_right ? min(i + off + right, Sk_b - 1) : Sk_b - 1; };
-  const int r_last = min(row0 + T * kBM - 1, Sq_b - 1);
-  const int k_begin = max(0, lo_of(row0));
-  const int k_end = hi_of(r_last) + 1;  // exclusive
-  const int j_lo = k_begin / kBN;
-  const int n_blk = (k_end > k_begin) ? (k_end + kBN - 1) / kBN - j_lo : 0;
 
   // ---------------------------------------------------------- shared memory
   uint8_t* sQ = smem + Cfg::kQOff;
@@ -220,11 +293,14 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
   uint64_t* drain = bars + 7 + 4 * ST;    // [2]: one per issuer
   uint64_t* s_free = bars + 9 + 4 * ST;   // softmax has S_t in registers (separate-P layout)
   uint64_t* pv_done = bars + 11 + 4 * ST; // PV_t finished: P_t may be rewritten, O_t rescaled
+  uint64_t* q_empty = bars + 13 + 4 * ST; // the last product reading this unit's Q is done
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
+  constexpr int kIssuers = Cfg::kSepP ? T : 1;
 
   if (warp == Cfg::kProducerWarp && lane == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, kIssuers);  // one commit per issuer
     for (int s = 0; s < ST; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(k_empty + s, T);  // released once per tile
@@ -253,82 +329,94 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
   const uint32_t tbase = *tmem_holder;
   const WaitCtx w{abort_flag, p.status, p.timeout_ns};
   const bool varlen = p.cu_q != nullptr;
-  const int b_coord = varlen ? 0 : b;
   if (warp >= Cfg::kProducerWarp) {
    regs_dec<Cfg::kOtherRegs>();
    if (warp == Cfg::kProducerWarp) {
     // ======================================================== TMA producer
-    if (lane == 0 && n_blk > 0) {
+    if (lane == 0) {
       tma_prefetch_map(&tmQ);
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
-      const int qrow = (varlen ? q0 : 0) + row0;
-      const int krow = varlen ? k0 : 0;
-      mbar_arrive_expect_tx(q_full, T * Cfg::kTileBytes);
-      for (int t = 0; t < T; ++t)
-        for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_4d(sQ + t * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmQ, q_full, c * Cfg::kChunkElems,
-                      qrow + t * kBM, h, b_coord);
+      int kv_it = 0;  // K/V blocks loaded so far: ring slot kv_it % ST
+      int q_cnt = 0;  // units whose Q tiles were loaded
       int last_k[ST], last_v[ST];
       for (int s = 0; s < ST; ++s) last_k[s] = last_v[s] = -1;
-      for (int it = 0; it < n_blk; ++it) {
-        const int s = it % ST;
-        const uint32_t ph = (it / ST) & 1;
-        const int j = j_lo + it;
-        if constexpr (!KV) {
-          if (!wait_bounded(k_empty + s, ph ^ 1, w)) break;
-          mbar_arrive_expect_tx(k_full + s, Cfg::kTileBytes);
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const FwdUnit u = fwd_unit_at<T, KV>(p, k);
+        if (u.state == 0) break;
+        if (u.state == 1 || u.n_blk == 0) continue;
+        const int b_coord = varlen ? 0 : u.b;
+        const int hk = u.h / p.G;
+        // the previous unit's Q stays in place until its last QK product has run
+        if (q_cnt > 0 && !(ok = wait_bounded(q_empty, (q_cnt - 1) & 1, w))) break;
+        const int qrow = (varlen ? u.q0 : 0) + u.row0;
+        const int krow = varlen ? u.k0 : 0;
+        mbar_arrive_expect_tx(q_full, T * Cfg::kTileBytes);
+        for (int t = 0; t < T; ++t)
           for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_4d(sK + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmK, k_full + s,
-                        c * Cfg::kChunkElems, krow + j * kBN, hk, b_coord);
-          last_k[s] = ph;
-          if (!wait_bounded(v_empty + s, ph ^ 1, w)) break;
-          mbar_arrive_expect_tx(v_full + s, Cfg::kTileBytes);
-          for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_4d(sV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmV, v_full + s,
-                        c * Cfg::kChunkElems, krow + j * kBN, hk, b_coord);
-          last_v[s] = ph;
-        } else {
-          // KV cache: the block's two 64-key halves, each inside one page (page_size
-          // is a multiple of 64); halves at or past the sequence's end are not
-          // loaded (their rows are masked, and V's are zeroed before P.V)
-          int row[2], blk[2], nh = 0;
-          for (int hh = 0; hh < 2; ++hh) {
-            const int pos = j * kBN + hh * 64;
-            if (pos >= Sk_b) break;
-            if (p.block_table != nullptr) {
-              int bk = p.block_table[static_cast<int64_t>(b) * p.max_blocks + pos / p.page_size];
-              if (bk < 0 || bk >= p.num_blocks) {
-                atomicOr(p.status, kDevBadBlock);
-                bk = 0;  // read a valid page; the status word reports the fault
+            tma_load_4d(sQ + t * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmQ, q_full,
+                        c * Cfg::kChunkElems, qrow + t * kBM, u.h, b_coord);
+        ++q_cnt;
+        for (int it = 0; it < u.n_blk; ++it, ++kv_it) {
+          const int s = kv_it % ST;
+          const uint32_t ph = (kv_it / ST) & 1;
+          const int j = u.j_lo + it;
+          if constexpr (!KV) {
+            if (!(ok = wait_bounded(k_empty + s, ph ^ 1, w))) break;
+            mbar_arrive_expect_tx(k_full + s, Cfg::kTileBytes);
+            for (int c = 0; c < Cfg::kChunks; ++c)
+              tma_load_4d(sK + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmK, k_full + s,
+                          c * Cfg::kChunkElems, krow + j * kBN, hk, b_coord);
+            last_k[s] = ph;
+            if (!(ok = wait_bounded(v_empty + s, ph ^ 1, w))) break;
+            mbar_arrive_expect_tx(v_full + s, Cfg::kTileBytes);
+            for (int c = 0; c < Cfg::kChunks; ++c)
+              tma_load_4d(sV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmV, v_full + s,
+                          c * Cfg::kChunkElems, krow + j * kBN, hk, b_coord);
+            last_v[s] = ph;
+          } else {
+            // KV cache: the block's two 64-key halves, each inside one page (page_size
+            // is a multiple of 64); halves at or past the sequence's end are not
+            // loaded (their rows are masked, and V's are zeroed before P.V)
+            int row[2], blk[2], nh = 0;
+            for (int hh = 0; hh < 2; ++hh) {
+              const int pos = j * kBN + hh * 64;
+              if (pos >= u.Sk_b) break;
+              if (p.block_table != nullptr) {
+                int bk = p.block_table[static_cast<int64_t>(u.b) * p.max_blocks + pos / p.page_size];
+                if (bk < 0 || bk >= p.num_blocks) {
+                  atomicOr(p.status, kDevBadBlock);
+                  bk = 0;  // read a valid page; the status word reports the fault
+                }
+                row[hh] = pos % p.page_size;
+                blk[hh] = bk;
+              } else {
+                row[hh] = pos;
+                blk[hh] = u.b;
               }
-              row[hh] = pos % p.page_size;
-              blk[hh] = bk;
-            } else {
-              row[hh] = pos;
-              blk[hh] = b;
+              ++nh;
             }
-            ++nh;
+            constexpr uint32_t kHalfBytes = Cfg::kChunks * 64 * 128;
+            if (!(ok = wait_bounded(k_empty + s, ph ^ 1, w))) break;
+            mbar_arrive_expect_tx(k_full + s, nh * kHalfBytes);
+            for (int hh = 0; hh < nh; ++hh)
+              for (int c = 0; c < Cfg::kChunks; ++c)
+                tma_load_4d(sK + s * Cfg::kTileBytes + c * Cfg::kChunkBytes + hh * 64 * 128, &tmK,
+                            k_full + s, c * Cfg::kChunkElems, row[hh], hk, blk[hh]);
+            last_k[s] = ph;
+            if (!(ok = wait_bounded(v_empty + s, ph ^ 1, w))) break;
+            mbar_arrive_expect_tx(v_full + s, nh * kHalfBytes);
+            for (int hh = 0; hh < nh; ++hh)
+              for (int c = 0; c < Cfg::kChunks; ++c)
+                tma_load_4d(sV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes + hh * 64 * 128, &tmV,
+                            v_full + s, c * Cfg::kChunkElems, row[hh], hk, blk[hh]);
+            last_v[s] = ph;
           }
-          constexpr uint32_t kHalfBytes = Cfg::kChunks * 64 * 128;
-          if (!wait_bounded(k_empty + s, ph ^ 1, w)) break;
-          mbar_arrive_expect_tx(k_full + s, nh * kHalfBytes);
-          for (int hh = 0; hh < nh; ++hh)
-            for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_4d(sK + s * Cfg::kTileBytes + c * Cfg::kChunkBytes + hh * 64 * 128, &tmK,
-                          k_full + s, c * Cfg::kChunkElems, row[hh], hk, blk[hh]);
-          last_k[s] = ph;
-          if (!wait_bounded(v_empty + s, ph ^ 1, w)) break;
-          mbar_arrive_expect_tx(v_full + s, nh * kHalfBytes);
-          for (int hh = 0; hh < nh; ++hh)
-            for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_4d(sV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes + hh * 64 * 128, &tmV,
-                          v_full + s, c * Cfg::kChunkElems, row[hh], hk, blk[hh]);
-          last_v[s] = ph;
         }
       }
       if (*abort_flag) {  // let this CTA's own copies land before the smem goes away
-        wait_drain(q_full, 0, p.timeout_ns);
+        if (q_cnt > 0) wait_drain(q_full, (q_cnt - 1) & 1, p.timeout_ns);
         for (int s = 0; s < ST; ++s) {
           if (last_k[s] >= 0) wait_drain(k_full + s, last_k[s], p.timeout_ns);
           if (last_v[s] >= 0) wait_drain(v_full + s, last_v[s], p.timeout_ns);
@@ -340,63 +428,85 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
     // ======================================================== MMA issuer (D = 128)
     // One thread alternates the tiles, PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so
     // one tile's softmax overlaps the other tile's products.
-    if (lane == 0 && n_blk > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_qk = f16_idesc(BF16 && !FP8, kBM, kBN, false, false);
       constexpr uint32_t idesc_pv = f16_idesc(BF16 && !FP8, kBM, D, false, true);
+      // K-major Q and K (leading offset 16 B) and MN-major V (leading offset one
+      // 16 KiB atom column) share the high descriptor word (stride offset 1 KiB)
       const uint64_t dQ0 = sw128_desc(smem_u32(sQ), 16, 1024);
-      const uint64_t dQ1 = desc_advance(dQ0, Cfg::kTileBytes);
-      const uint64_t dK = sw128_desc(smem_u32(sK), 16, 1024);
-      const uint64_t dV = sw128_desc(smem_u32(sV), Cfg::kChunkBytes, 1024);
-#define FA_QK(T, S)                                                                    \
-  fwd_issue_qk<D, E>(tbase + (T) * kBM, (T) ? dQ1 : dQ0,                                    \
-                  desc_advance(dK, (S) * Cfg::kTileBytes), idesc_qk)
-#define FA_PV(T, S, ACC)                                                               \
+      const uint64_t dV0 = sw128_desc(smem_u32(sV), Cfg::kChunkBytes, 1024);
+      const uint32_t hi = static_cast<uint32_t>(dQ0 >> 32);
+      const uint32_t q_lo = static_cast<uint32_t>(dQ0);
+      const uint32_t k_lo = static_cast<uint32_t>(sw128_desc(smem_u32(sK), 16, 1024));
+      const uint32_t v_lo = static_cast<uint32_t>(dV0);
+      constexpr uint32_t kTileStep = Cfg::kTileBytes >> 4;
+#define FA_QK(T, S)                                                                        \
+  fwd_issue_qk<D, E>(tbase + (T) * kBM, q_lo + (T) * kTileStep, k_lo + (S) * kTileStep, hi, \
+                     idesc_qk)
+#define FA_PV(T, S, ACC)                                                                   \
   fwd_issue_pv<D, E>(tbase + Cfg::kOCol + (T) * D, tbase + Cfg::kPCol + (T) * Cfg::kPStride, \
-                  desc_advance(dV, (S) * Cfg::kTileBytes), idesc_pv, ACC)
-      bool ok = wait_bounded(q_full, 0, w) && wait_bounded(k_full, 0, w);
-      if (ok) {
+                     v_lo + (S) * kTileStep, hi, idesc_pv, ACC)
+      int kv_it = 0;  // ring position of the unit's first block
+      int blk = 0;    // blocks completed per tile so far: s_full / p_full phases
+      int q_cnt = 0;  // units started: q_full phase
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const FwdUnit u = fwd_unit_at<T, KV>(p, k);
+        if (u.state == 0) break;
+        if (u.state == 1 || u.n_blk == 0) continue;
+        const int n = u.n_blk;
+        ok = wait_bounded(q_full, q_cnt & 1, w) &&
+             wait_bounded(k_full + kv_it % ST, (kv_it / ST) & 1, w);
+        if (!ok) break;
         tc_fence_after();
-        FA_QK(0, 0);
+        FA_QK(0, kv_it % ST);
         tc_commit(s_full + 0);
-        FA_QK(1, 0);
+        FA_QK(1, kv_it % ST);
         tc_commit(s_full + 1);
-        tc_commit(k_empty + 0);
-        tc_commit(k_empty + 0);  // k_empty counts one release per tile
-      }
-      for (int it = 0; it < n_blk && ok; ++it) {
-        const int s = it % ST;
-        const uint32_t ph = (it / ST) & 1;
-        const bool more = it + 1 < n_blk;
-        const int s1 = (it + 1) % ST;
-        const uint32_t ph1 = ((it + 1) / ST) & 1;
-        if (!(ok = wait_bounded(v_full + s, ph, w))) break;
-        if (!(ok = wait_bounded(p_full + 0, it & 1, w))) break;
-        tc_fence_after();
-        FA_PV(0, s, it > 0);
-        tc_commit(v_empty + s);
-        if (more) {
-          if (!(ok = wait_bounded(k_full + s1, ph1, w))) break;
+        tc_commit(k_empty + kv_it % ST);
+        tc_commit(k_empty + kv_it % ST);  // k_empty counts one release per tile
+        if (n == 1) tc_commit(q_empty);
+        for (int it = 0; it < n; ++it) {
+          const int g = kv_it + it;
+          const int s = g % ST;
+          const uint32_t ph = (g / ST) & 1;
+          const bool more = it + 1 < n;
+          const int s1 = (g + 1) % ST;
+          const uint32_t ph1 = ((g + 1) / ST) & 1;
+          const uint32_t pp = (blk + it) & 1;
+          if (!(ok = wait_bounded(v_full + s, ph, w))) break;
+          if (!(ok = wait_bounded(p_full + 0, pp, w))) break;
           tc_fence_after();
-          FA_QK(0, s1);
-          tc_commit(s_full + 0);
-          tc_commit(k_empty + s1);
-        } else {
-          tc_commit(o_final + 0);
+          FA_PV(0, s, it > 0);
+          tc_commit(v_empty + s);
+          if (more) {
+            if (!(ok = wait_bounded(k_full + s1, ph1, w))) break;
+            tc_fence_after();
+            FA_QK(0, s1);
+            tc_commit(s_full + 0);
+            tc_commit(k_empty + s1);
+          } else {
+            tc_commit(o_final + 0);
+          }
+          if (!(ok = wait_bounded(p_full + 1, pp, w))) break;
+          tc_fence_after();
+          FA_PV(1, s, it > 0);
+          tc_commit(v_empty + s);
+          if (more) {
+            FA_QK(1, s1);
+            tc_commit(s_full + 1);
+            tc_commit(k_empty + s1);
+            if (it + 2 == n) tc_commit(q_empty);  // that was the unit's last QK
+          } else {
+            tc_commit(o_final + 1);
+          }
         }
-        if (!(ok = wait_bounded(p_full + 1, it & 1, w))) break;
-        tc_fence_after();
-        FA_PV(1, s, it > 0);
-        tc_commit(v_empty + s);
-        if (more) {
-          FA_QK(1, s1);
-          tc_commit(s_full + 1);
-          tc_commit(k_empty + s1);
-        } else {
-          tc_commit(o_final + 1);
-        }
-      }
 #undef FA_QK
 #undef FA_PV
+        kv_it += n;
+        blk += n;
+        ++q_cnt;
+      }
       tc_commit(drain + 0);
       wait_drain(drain + 0, 0, p.timeout_ns);
     }
@@ -404,50 +514,67 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
    } else if (Cfg::kSepP && warp >= Cfg::kIssuerWarp && warp < Cfg::kIssuerWarp + T) {
     // ======================================================== MMA issuers (D = 64)
     const int t = warp - Cfg::kIssuerWarp;  // this issuer's query tile
-    if (lane == 0 && n_blk > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_qk = f16_idesc(BF16 && !FP8, kBM, kBN, false, false);
       constexpr uint32_t idesc_pv = f16_idesc(BF16 && !FP8, kBM, D, false, true);
       const uint32_t tS = tbase + t * kBM;
       const uint32_t tP = tbase + Cfg::kPCol + t * Cfg::kPStride;
       const uint32_t tO = tbase + Cfg::kOCol + t * D;
-      const uint64_t dQ = desc_advance(sw128_desc(smem_u32(sQ), 16, 1024), t * Cfg::kTileBytes);
-      const uint64_t dK = sw128_desc(smem_u32(sK), 16, 1024);               // K-major
-      const uint64_t dV = sw128_desc(smem_u32(sV), Cfg::kChunkBytes, 1024); // MN-major
-#define FA_QK(S) fwd_issue_qk<D, E>(tS, dQ, desc_advance(dK, (S) * Cfg::kTileBytes), idesc_qk)
-#define FA_PV(S, ACC) \
-  fwd_issue_pv<D, E>(tO, tP, desc_advance(dV, (S) * Cfg::kTileBytes), idesc_pv, ACC)
-      bool ok = wait_bounded(q_full, 0, w) && wait_bounded(k_full, 0, w);
-      if (ok) {
+      constexpr uint32_t kTileStep = Cfg::kTileBytes >> 4;
+      const uint64_t dQ0 = sw128_desc(smem_u32(sQ), 16, 1024);                  // K-major
+      const uint32_t hi = static_cast<uint32_t>(dQ0 >> 32);  // shared by Q, K and V
+      const uint32_t q_lo = static_cast<uint32_t>(dQ0) + t * kTileStep;
+      const uint32_t k_lo = static_cast<uint32_t>(sw128_desc(smem_u32(sK), 16, 1024));
+      const uint32_t v_lo = static_cast<uint32_t>(sw128_desc(smem_u32(sV), Cfg::kChunkBytes, 1024));
+#define FA_QK(S) fwd_issue_qk<D, E>(tS, q_lo, k_lo + (S) * kTileStep, hi, idesc_qk)
+#define FA_PV(S, ACC) fwd_issue_pv<D, E>(tO, tP, v_lo + (S) * kTileStep, hi, idesc_pv, ACC)
+      int kv_it = 0, blk = 0, q_cnt = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const FwdUnit u = fwd_unit_at<T, KV>(p, k);
+        if (u.state == 0) break;
+        if (u.state == 1 || u.n_blk == 0) continue;
+        const int n = u.n_blk;
+        ok = wait_bounded(q_full, q_cnt & 1, w) &&
+             wait_bounded(k_full + kv_it % ST, (kv_it / ST) & 1, w);
+        if (!ok) break;
         tc_fence_after();
-        FA_QK(0);
+        FA_QK(kv_it % ST);
         tc_commit(s_full + t);
-        tc_commit(k_empty + 0);
-      }
-      for (int it = 0; it < n_blk && ok; ++it) {
-        const int s = it % ST;
-        const uint32_t ph = (it / ST) & 1;
-        const bool more = it + 1 < n_blk;
-        const int s1 = (it + 1) % ST;
-        const uint32_t ph1 = ((it + 1) / ST) & 1;
-        // QK_t(j+1) as soon as softmax t holds S_t(j) in registers
-        if (more) {
-          if (!(ok = wait_bounded(k_full + s1, ph1, w))) break;
-          if (!(ok = wait_bounded(s_free + t, it & 1, w))) break;
+        tc_commit(k_empty + kv_it % ST);
+        if (n == 1) tc_commit(q_empty);
+        for (int it = 0; it < n; ++it) {
+          const int g = kv_it + it;
+          const int s = g % ST;
+          const uint32_t ph = (g / ST) & 1;
+          const bool more = it + 1 < n;
+          const int s1 = (g + 1) % ST;
+          const uint32_t ph1 = ((g + 1) / ST) & 1;
+          const uint32_t pp = (blk + it) & 1;
+          // QK_t(j+1) as soon as softmax t holds S_t(j) in registers
+          if (more) {
+            if (!(ok = wait_bounded(k_full + s1, ph1, w))) break;
+            if (!(ok = wait_bounded(s_free + t, pp, w))) break;
+            tc_fence_after();
+            FA_QK(s1);
+            tc_commit(s_full + t);
+            tc_commit(k_empty + s1);
+            if (it + 2 == n) tc_commit(q_empty);  // that was the unit's last QK
+          }
+          if (!(ok = wait_bounded(v_full + s, ph, w))) break;
+          if (!(ok = wait_bounded(p_full + t, pp, w))) break;
           tc_fence_after();
-          FA_QK(s1);
-          tc_commit(s_full + t);
-          tc_commit(k_empty + s1);
+          FA_PV(s, it > 0);
+          tc_commit(pv_done + t);
+          tc_commit(v_empty + s);
+          if (!more) tc_commit(o_final + t);
         }
-        if (!(ok = wait_bounded(v_full + s, ph, w))) break;
-        if (!(ok = wait_bounded(p_full + t, it & 1, w))) break;
-        tc_fence_after();
-        FA_PV(s, it > 0);
-        tc_commit(pv_done + t);
-        tc_commit(v_empty + s);
-        if (!more) tc_commit(o_final + t);
-      }
 #undef FA_QK
 #undef FA_PV
+        kv_it += n;
+        blk += n;
+        ++q_cnt;
+      }
       // every MMA issued above is complete before tensor memory is released
       tc_commit(drain + t);
       wait_drain(drain + t, 0, p.timeout_ns);
@@ -463,21 +590,35 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
     const uint32_t tS = tbase + t * kBM + lane_off;
     const uint32_t tP = tbase + Cfg::kPCol + t * Cfg::kPStride + lane_off;
     const uint32_t tO = tbase + Cfg::kOCol + t * D + lane_off;
-    const int i = row0 + t * kBM + r;  // query row within the sequence
-    const int ra = row0 + t * kBM;
+    int blk = 0;    // blocks of this tile so far: s_full / pv_done phases
+    int u_cnt = 0;  // units with at least one block: o_final phase
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+    const FwdUnit u = fwd_unit_at<T, KV>(p, k);
+    if (u.state == 0) break;
+    if (u.state == 1) continue;
+    const int off = u.off, Sq_b = u.Sq_b, Sk_b = u.Sk_b, h = u.h;
+    const int j_lo = u.j_lo, n_blk = u.n_blk;
+    const bool has_left = p.wl >= 0;
+    const bool has_right = p.causal || p.wr >= 0;
+    const int right = p.causal ? 0 : p.wr;
+    // allowed keys of row i: [lo(i), hi(i)] intersected with [0, Sk_b)
+    auto lo_of = [&](int i) { return has_left ? i + off - p.wl : INT_MIN / 2; };
+    auto hi_of = [&](int i) { return has_right ? min(i + off + right, Sk_b - 1) : Sk_b - 1; };
+    const int i = u.row0 + t * kBM + r;  // query row within the sequence
+    const int ra = u.row0 + t * kBM;
     const int rb = max(ra, min(ra + kBM - 1, Sq_b - 1));
     const int lo_i = lo_of(i), hi_i = hi_of(i);
     const int lo_rb = lo_of(rb), hi_ra = hi_of(ra);
     const float slope2 = ALIBI ? p.alibi[h] * kLog2e : 0.f;
     const float ipo = static_cast<float>(i + off);
     float m_use = -INFINITY;  // running max, base-2 units
-    float l = 0.f;            // running sum of exp2(x - m_use): gives the LSE
-    float lr = 0.f;           // the same sum over P rounded to 16 bits: normalises O
-    bool ok = true;
+    float l = 0.f;            // running sum of exp2(x - m_use): the LSE and O's normaliser
 
     for (int it = 0; it < n_blk; ++it) {
       const int kb = (j_lo + it) * kBN;
-      ok = wait_bounded(s_full + t, it & 1, w);
+      const uint32_t pp = (blk + it) & 1;
+      ok = wait_bounded(s_full + t, pp, w);
       if (!__all_sync(0xffffffffu, ok)) {  // keep the warp's .sync.aligned ops uniform
         ok = false;
         break;
@@ -493,7 +634,6 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free + t);
       }
-
       const bool masked = (kb < lo_rb) || (kb + kBN - 1 > hi_ra);
       const int lo_c = lo_i - kb, hi_c = hi_i - kb;  // allowed columns: lo_c <= c <= hi_c
       float factor;  // exponent argument = s * factor - m
@@ -501,9 +641,21 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
         // raw-score domain: mask here, fold the scale into the exponent below
         // (softmax_scale > 0 here: the host maps 0 to a tiny positive scale)
         if (masked) {
+          // test only the bounds that cut into this block for some row of the warp
+          // (a causal diagonal block has only the right one)
+          const bool cut_lo = __any_sync(0xffffffffu, lo_c > 0);
+          const bool cut_hi = __any_sync(0xffffffffu, hi_c < kBN - 1);
+          constexpr uint32_t kNegInf = 0xFF800000u;
+          if (cut_lo && cut_hi) {
 #pragma unroll
-          for (int c = 0; c < kBN; ++c)
-            s[c] = (c >= lo_c && c <= hi_c) ? s[c] : __float_as_uint(-INFINITY);
+            for (int c = 0; c < kBN; ++c) s[c] = (c >= lo_c && c <= hi_c) ? s[c] : kNegInf;
+          } else if (cut_hi) {
+#pragma unroll
+            for (int c = 0; c < kBN; ++c) s[c] = (c <= hi_c) ? s[c] : kNegInf;
+          } else if (cut_lo) {
+#pragma unroll
+            for (int c = 0; c < kBN; ++c) s[c] = (c >= lo_c) ? s[c] : kNegInf;
+          }
         }
         factor = p.scale_log2;
       } else {
@@ -564,7 +716,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
       // and the wait for PV_t(j-1) (which still reads P_t) comes only before the
       // stores, so the exponentials overlap it; with P aliasing S each 32-column
       // chunk is stored as soon as it is ready.
-      float2 lsum[kBN / 32], lrnd[kBN / 32];
+      float2 lsum[kBN / 32];
       uint32_t pk[Cfg::kSepP ? kBN / 2 : 16];
       auto exps = [&](auto with_max) {
         constexpr bool kMax = decltype(with_max)::value;
@@ -574,7 +726,6 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
 #pragma unroll
         for (int q4 = 0; q4 < kBN / 32; ++q4) {
           lsum[q4] = make_float2(0.f, 0.f);
-          lrnd[q4] = make_float2(0.f, 0.f);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const float s0 = __uint_as_float(s[q4 * 32 + 2 * e]);
@@ -599,10 +750,10 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
                 pk[e / 2] = pack4_e4m3(prev.x, prev.y, pp.x, pp.y);
             } else {
               const int pi = Cfg::kSepP ? q4 * 16 + e : e;
+              // P is rounded to 16 bits for the PV product while l sums the fp32
+              // values: O / l then carries at most the rounding's relative error
+              // (2^-9 for bf16, 2^-11 for fp16) on top of the output's own rounding
               pk[pi] = pack2<BF16>(pp.x, pp.y);
-              // bf16 P is rounded by up to 2^-9: sum the rounded values the PV
-              // product uses, so that O / lr is an exact convex combination of V rows
-              if constexpr (BF16) lrnd[q4] = add2(lrnd[q4], unpack2<true>(pk[pi]));
             }
           }
           if constexpr (FP8)
@@ -619,11 +770,10 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
         exps(std::false_type{});
       }
       l *= alpha;
-      lr *= alpha;
       if constexpr (Cfg::kSepP) {
         // P_t(j-1) must have been consumed (and O_t updated) by PV_t(j-1)
         if (it > 0) {
-          ok = wait_bounded(pv_done + t, (it - 1) & 1, w);
+          ok = wait_bounded(pv_done + t, (blk + it - 1) & 1, w);
           if (!__all_sync(0xffffffffu, ok)) {
             ok = false;
             break;
@@ -634,10 +784,8 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
         for (int q4 = 0; q4 < kBN / 32; ++q4) tmem_st16(tP + q4 * 16, pk + q4 * 16);
       }
       {
-        float2 a = add2(add2(lsum[0], lsum[1]), add2(lsum[2], lsum[3]));
+        const float2 a = add2(add2(lsum[0], lsum[1]), add2(lsum[2], lsum[3]));
         l += a.x + a.y;
-        if constexpr (BF16 && !FP8) a = add2(add2(lrnd[0], lrnd[1]), add2(lrnd[2], lrnd[3]));
-        lr += a.x + a.y;
       }
       // O_t rescale (after the score row is dead: lower register peak); it only
       // has to land before P_t is released to the MMA warp
@@ -657,8 +805,8 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
       // NaN in P.V, so this warp zeroes its 32 rows of them before releasing P
       // (both tiles' warps write the same zeros)
       if (KV && kb + kBN > Sk_b) {
-        const int s = it % ST;
-        ok = wait_bounded(v_full + s, (it / ST) & 1, w);
+        const int s = (blk + it) % ST;
+        ok = wait_bounded(v_full + s, ((blk + it) / ST) & 1, w);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
@@ -680,20 +828,20 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
     }
 
     // ---- epilogue: O / l -> 16-bit, LSE (natural log)
-    if (ok && n_blk > 0) ok = wait_bounded(o_final + t, 0, w);
+    if (ok && n_blk > 0) ok = wait_bounded(o_final + t, u_cnt & 1, w);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
       const bool row_ok = i < Sq_b;
       // a row with no allowed key keeps m = -inf (its sum may hold clamped
       // polynomial exponentials of -inf, each <= 2^-126): O = 0, LSE = -inf
-      const bool dead = (m_use == -INFINITY) || !(lr > 0.f);
+      const bool dead = (m_use == -INFINITY) || !(l > 0.f);
       // 8-bit inputs: O carries V's descale factor (Q's and K's sit in the scale)
-      const float inv = dead ? 0.f : (FP8 ? p.v_descale : 1.f) / lr;
+      const float inv = dead ? 0.f : (FP8 ? p.v_descale : 1.f) / l;
       uint8_t* orow = nullptr;
       if (row_ok) {
-        const int64_t ro = varlen ? static_cast<int64_t>(q0 + i) * p.o_ss
-                                  : static_cast<int64_t>(b) * p.o_sb +
+        const int64_t ro = varlen ? static_cast<int64_t>(u.q0 + i) * p.o_ss
+                                  : static_cast<int64_t>(u.b) * p.o_sb +
                                         static_cast<int64_t>(i) * p.o_ss;
         orow = static_cast<uint8_t*>(p.out) + (ro + static_cast<int64_t>(h) * p.o_sh) * 2;
       }
@@ -721,11 +869,14 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
       if (row_ok && p.lse != nullptr) {
         const float lse =
             dead ? -INFINITY : (m_use - (FP8 ? kP8Offset : 0.f) + __log2f(l)) * kLn2;
-        const int64_t li = varlen ? static_cast<int64_t>(h) * p.total_q + q0 + i
-                                  : (static_cast<int64_t>(b) * p.H + h) * p.Sq + i;
+        const int64_t li = varlen ? static_cast<int64_t>(h) * p.total_q + u.q0 + i
+                                  : (static_cast<int64_t>(u.b) * p.H + h) * p.Sq + i;
         p.lse[li] = lse;
       }
     }
+    blk += n_blk;
+    if (n_blk > 0) ++u_cnt;
+    }  // units
   }
 
   // ---------------------------------------------------------- teardown

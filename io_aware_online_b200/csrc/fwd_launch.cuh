@@ -2,6 +2,7 @@
 // dtype (included by fwd_f16.cu and fwd_bf16.cu so the two compile in parallel).
 #pragma once
 
+#include <algorithm>
 #include <cstdlib>
 
 #include "fwd_kernel.cuh"
@@ -21,10 +22,19 @@ cudaError_t launch_fwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const 
                              cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   const int n_units = (rows_q + T * kBM - 1) / (T * kBM);
-  const dim3 grid = p.tile_major ? dim3(static_cast<unsigned>(n_units), static_cast<unsigned>(p.H),
-                                         static_cast<unsigned>(batch))
-                                  : dim3(static_cast<unsigned>(p.H), static_cast<unsigned>(batch),
-                                         static_cast<unsigned>(n_units));
+  dim3 grid;
+  if (p.persistent) {
+    // as many CTAs as are resident at once (Cfg::kMinBlocks per SM), or fewer items
+    const long n_pi = p.pair ? (n_units + 1) / 2 : n_units;
+    const long items = static_cast<long>(batch) * p.H * n_pi;
+    const long slots = static_cast<long>(p.sm_count) * Cfg::kMinBlocks;
+    grid = dim3(static_cast<unsigned>(std::max(1L, std::min(items, slots))));
+  } else {
+    grid = p.tile_major ? dim3(static_cast<unsigned>(n_units), static_cast<unsigned>(p.H),
+                               static_cast<unsigned>(batch))
+                        : dim3(static_cast<unsigned>(p.H), static_cast<unsigned>(batch),
+                               static_cast<unsigned>(n_units));
+  }
   kern<<<grid, Cfg::kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }

@@ -235,6 +235,16 @@ __device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) 
   return (desc & 0xFFFFFFFF00000000ull) | lo;
 }
 
+// A 64-bit descriptor from its two 32-bit halves, built at the point of use: the
+// volatile asm keeps the compiler from hoisting every advanced descriptor of an
+// unrolled issue sequence out of the loop around it (which costs two registers
+// each in a warp that runs with few).
+__device__ __forceinline__ uint64_t desc_pack(uint32_t lo, uint32_t hi) {
+  uint64_t d;
+  asm volatile("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+  return d;
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16 with fp32 accumulation.
 // a_mn / b_mn select the MN-major (transposed) operand layouts.
 __host__ __device__ constexpr uint32_t f16_idesc(bool bf16, int M, int N, bool a_mn, bool b_mn) {
