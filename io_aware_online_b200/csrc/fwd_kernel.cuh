@@ -594,29 +594,40 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
     int u_cnt = 0;  // units with at least one block: o_final phase
     bool ok = true;
     for (int k = 0; ok; ++k) {
-    const FwdUnit u = fwd_unit_at<T, KV>(p, k);
-    if (u.state == 0) break;
-    if (u.state == 1) continue;
-    const int off = u.off, Sq_b = u.Sq_b, Sk_b = u.Sk_b, h = u.h;
-    const int j_lo = u.j_lo, n_blk = u.n_blk;
-    const bool has_left = p.wl >= 0;
-    const bool has_right = p.causal || p.wr >= 0;
-    const int right = p.causal ? 0 : p.wr;
-    // allowed keys of row i: [lo(i), hi(i)] intersected with [0, Sk_b)
-    auto lo_of = [&](int i) { return has_left ? i + off - p.wl : INT_MIN / 2; };
-    auto hi_of = [&](int i) { return has_right ? min(i + off + right, Sk_b - 1) : Sk_b - 1; };
-    const int i = u.row0 + t * kBM + r;  // query row within the sequence
-    const int ra = u.row0 + t * kBM;
-    const int rb = max(ra, min(ra + kBM - 1, Sq_b - 1));
-    const int lo_i = lo_of(i), hi_i = hi_of(i);
-    const int lo_rb = lo_of(rb), hi_ra = hi_of(ra);
-    const float slope2 = ALIBI ? p.alibi[h] * kLog2e : 0.f;
-    const float ipo = static_cast<float>(i + off);
+    // what the block loop needs of the unit; the epilogue looks the unit up again
+    // (fewer values live across the loop next to the 128-float score row)
+    int kb0, n_blk, lo_i, hi_i, lo_rb, hi_ra, Sk_b;
+    float slope2, ipo;
+    {
+      const FwdUnit u = fwd_unit_at<T, KV>(p, k);
+      if (u.state == 0) break;
+      if (u.state == 1) continue;
+      const int off = u.off, Sq_b = u.Sq_b;
+      Sk_b = u.Sk_b;
+      kb0 = u.j_lo * kBN;
+      n_blk = u.n_blk;
+      const bool has_left = p.wl >= 0;
+      const bool has_right = p.causal || p.wr >= 0;
+      const int right = p.causal ? 0 : p.wr;
+      // allowed keys of row i: [lo(i), hi(i)] intersected with [0, Sk_b)
+      auto lo_of = [&](int i) { return has_left ? i + off - p.wl : INT_MIN / 2; };
+      auto hi_of = [&](int i) { return has_right ? min(i + off + right, Sk_b - 1) : Sk_b - 1; };
+      const int i = u.row0 + t * kBM + r;  // query row within the sequence
+      const int ra = u.row0 + t * kBM;
+      const int rb = max(ra, min(ra + kBM - 1, Sq_b - 1));
+      lo_i = lo_of(i);
+      hi_i = hi_of(i);
+      lo_rb = lo_of(rb);
+      hi_ra = hi_of(ra);
+      slope2 = ALIBI ? p.alibi[u.h] * kLog2e : 0.f;
+      ipo = static_cast<float>(i + off);
+    }
     float m_use = -INFINITY;  // running max, base-2 units
-    float l = 0.f;            // running sum of exp2(x - m_use): the LSE and O's normaliser
+    float l = 0.f;            // running sum of exp2(x - m_use): gives the LSE
+    float lr = 0.f;           // the same sum over P rounded to bf16: normalises O (bf16 only)
 
     for (int it = 0; it < n_blk; ++it) {
-      const int kb = (j_lo + it) * kBN;
+      const int kb = kb0 + it * kBN;
       const uint32_t pp = (blk + it) & 1;
       ok = wait_bounded(s_full + t, pp, w);
       if (!__all_sync(0xffffffffu, ok)) {  // keep the warp's .sync.aligned ops uniform
@@ -716,16 +727,21 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
       // and the wait for PV_t(j-1) (which still reads P_t) comes only before the
       // stores, so the exponentials overlap it; with P aliasing S each 32-column
       // chunk is stored as soon as it is ready.
-      float2 lsum[kBN / 32];
-      uint32_t pk[Cfg::kSepP ? kBN / 2 : 16];
-      auto exps = [&](auto with_max) {
+      // With separate P columns the first half of the row is computed before the
+      // wait for PV_t(j-1) (which still reads P_t) and held in registers; the second
+      // half is stored chunk by chunk as it is produced.  With P aliasing S every
+      // 32-column chunk is stored as soon as it is ready.
+      float2 lsum[kBN / 32], lrnd[kBN / 32];
+      uint32_t pk[Cfg::kSepP ? 32 : 16];
+      auto exps = [&](auto with_max, auto q_from, auto q_to) {
         constexpr bool kMax = decltype(with_max)::value;
         const float neg_m = (m_use == -INFINITY) ? 0.f : (FP8 ? kP8Offset : 0.f) - m_use;
         const float2 f2 = make_float2(factor, factor), nm2 = make_float2(neg_m, neg_m);
         float2 prev = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int q4 = 0; q4 < kBN / 32; ++q4) {
+        for (int q4 = decltype(q_from)::value; q4 < decltype(q_to)::value; ++q4) {
           lsum[q4] = make_float2(0.f, 0.f);
+          lrnd[q4] = make_float2(0.f, 0.f);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const float s0 = __uint_as_float(s[q4 * 32 + 2 * e]);
@@ -749,28 +765,27 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
               else
                 pk[e / 2] = pack4_e4m3(prev.x, prev.y, pp.x, pp.y);
             } else {
-              const int pi = Cfg::kSepP ? q4 * 16 + e : e;
-              // P is rounded to 16 bits for the PV product while l sums the fp32
-              // values: O / l then carries at most the rounding's relative error
-              // (2^-9 for bf16, 2^-11 for fp16) on top of the output's own rounding
+              const int pi = Cfg::kSepP ? (q4 % 2) * 16 + e : e;
               pk[pi] = pack2<BF16>(pp.x, pp.y);
+              // bf16 P is rounded by up to 2^-9: O is normalised by the sum of the
+              // rounded values the PV product uses, so that O / lr is an exact convex
+              // combination of V rows (fp16's 2^-11 rounding needs no such sum)
+              if constexpr (BF16) lrnd[q4] = add2(lrnd[q4], unpack2<true>(pk[pi]));
             }
           }
           if constexpr (FP8)
             tmem_st8(tP + q4 * 8, pk);
           else if constexpr (!Cfg::kSepP)
             tmem_st16(tP + q4 * 16, pk);
+          else if (q4 >= 2)
+            tmem_st16(tP + q4 * 16, pk + (q4 % 2) * 16);
         }
       };
-      if (spec) {
-        exps(std::true_type{});
-        update_max(fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * factor);
-        if (__any_sync(0xffffffffu, need)) exps(std::false_type{});
-      } else {
-        exps(std::false_type{});
-      }
-      l *= alpha;
+      using Q0 = std::integral_constant<int, 0>;
+      using Q2 = std::integral_constant<int, kBN / 64>;
+      using Q4 = std::integral_constant<int, kBN / 32>;
       if constexpr (Cfg::kSepP) {
+        exps(std::false_type{}, Q0{}, Q2{});
         // P_t(j-1) must have been consumed (and O_t updated) by PV_t(j-1)
         if (it > 0) {
           ok = wait_bounded(pv_done + t, (blk + it - 1) & 1, w);
@@ -780,24 +795,37 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
           }
           tc_fence_after();
         }
-#pragma unroll
-        for (int q4 = 0; q4 < kBN / 32; ++q4) tmem_st16(tP + q4 * 16, pk + q4 * 16);
+        tmem_st16(tP, pk);
+        tmem_st16(tP + 16, pk + 16);
+        exps(std::false_type{}, Q2{}, Q4{});
+      } else if (spec) {
+        exps(std::true_type{}, Q0{}, Q4{});
+        update_max(fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * factor);
+        if (__any_sync(0xffffffffu, need)) exps(std::false_type{}, Q0{}, Q4{});
+      } else {
+        exps(std::false_type{}, Q0{}, Q4{});
       }
+      l *= alpha;
+      if constexpr (BF16 && !FP8) lr *= alpha;
       {
         const float2 a = add2(add2(lsum[0], lsum[1]), add2(lsum[2], lsum[3]));
         l += a.x + a.y;
+        if constexpr (BF16 && !FP8) {
+          const float2 b = add2(add2(lrnd[0], lrnd[1]), add2(lrnd[2], lrnd[3]));
+          lr += b.x + b.y;
+        }
       }
       // O_t rescale (after the score row is dead: lower register peak); it only
       // has to land before P_t is released to the MMA warp
       if (__any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_ld_wait(o);
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t o[16];
+          tmem_ld16(tO + c * 16, o);
+          tmem_ld_wait16(o);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + c * 32, o);
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st16(tO + c * 16, o);
         }
       }
       // KV cache, last block of the sequence: V rows past its end hold whatever
@@ -832,12 +860,16 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
+      const FwdUnit u = fwd_unit_at<T, KV>(p, k);
+      const int i = u.row0 + t * kBM + r;
+      const int Sq_b = u.Sq_b, h = u.h;
       const bool row_ok = i < Sq_b;
       // a row with no allowed key keeps m = -inf (its sum may hold clamped
       // polynomial exponentials of -inf, each <= 2^-126): O = 0, LSE = -inf
-      const bool dead = (m_use == -INFINITY) || !(l > 0.f);
+      const float norm = (BF16 && !FP8) ? lr : l;
+      const bool dead = (m_use == -INFINITY) || !(norm > 0.f);
       // 8-bit inputs: O carries V's descale factor (Q's and K's sit in the scale)
-      const float inv = dead ? 0.f : (FP8 ? p.v_descale : 1.f) / l;
+      const float inv = dead ? 0.f : (FP8 ? p.v_descale : 1.f) / norm;
       uint8_t* orow = nullptr;
       if (row_ok) {
         const int64_t ro = varlen ? static_cast<int64_t>(u.q0 + i) * p.o_ss
@@ -846,24 +878,23 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
         orow = static_cast<uint8_t*>(p.out) + (ro + static_cast<int64_t>(h) * p.o_sh) * 2;
       }
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t o[16];
         if (n_blk > 0) {
-          tmem_ld32(tO + c * 32, o);
-          tmem_ld_wait(o);
+          tmem_ld16(tO + c * 16, o);
+          tmem_ld_wait16(o);
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
+          for (int e = 0; e < 16; ++e) o[e] = 0u;
         }
-        uint32_t pk[16];
+        uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
+        for (int e = 0; e < 8; ++e)
           pk[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
         if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
       if (row_ok && p.lse != nullptr) {
