@@ -19,6 +19,7 @@ combine(out_partial, lse_partial)          LSE-weighted combine of split partial
 append(kcache, vcache, k_new, v_new, cache_seqlens, block_table=None)
                                            KV-cache append (returns updated copies)
 attention_backward(q, k, v, do, ...)       gradients dq, dk, dv (backward.py, numpy fp64)
+attention_backward_varlen(q, k, v, do, cu_q, cu_k, ...)  the same over packed sequences
 """
 from __future__ import annotations
 
@@ -227,4 +228,4 @@ def append(kcache, vcache, k_new, v_new, cache_seqlens, block_table=None):
     return kc, vc
 
 
-from .backward import attention_backward  # noqa: E402,F401  (fp64 gradients; see backward.py)
+from .backward import attention_backward, attention_backward_varlen  # noqa: E402,F401  (fp64 gradients; see backward.py)
