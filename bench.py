@@ -4,13 +4,16 @@ One step = one pass of the whole path over one batch of synthetic input:
   1. prefill forward (fa_fwd): causal, B=4, S=4096, H=32, d=64, fp16
   2. paged split-KV decode (fa_fwd_kvcache) + LSE combine: B=64, Sq=1, H=32,
      Hkv=8, d=128, bf16, cache lengths U{1K..32K}, pages of 256, random
-     block_table, num_splits (default 16)
+     block_table, at num_splits 4 (headline), 16 and 1 (the unsplit control)
+Each kernel runs R times back to back per step (its inputs exceed the L2); the
+L2 is flushed between steps.  Per kernel the median and the minimum launch time
+over the steps are reported; ``value`` uses the median.
 Reported: ``value`` = prefill TFLOPS (4*d*sum of allowed (i, j) pairs / time);
 ``decode`` = KV-cache GB/s (valid cache bytes + q/out/lse/block_table / time).
 Both are also given as fractions of the measured B200 peaks.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-       [--num-splits S] [--no-cpu-baseline] [--no-e2e]
+       [--num-splits S] [--repeat R] [--no-cpu-baseline] [--no-e2e]
 For N > 1 launch under torch.distributed.run; every rank runs an independent
 replica on its own seeded data (weak scaling, no collective on the data path);
 the step time is the max over ranks.
@@ -76,6 +79,15 @@ def load_peaks():
             pk = json.load(f)
         return pk["hbm_gbs"], pk["bf16_tflops"], "measured"
     return 6650.0, 1590.0, "fallback"
+
+
+def sustained_tflops():
+    """The measured bf16 GEMM rate under the power cap (seconds-long loop), or None."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f).get("bf16_tflops_sustained")
+    return None
 
 
 class Clocks:
@@ -189,13 +201,19 @@ def make_decode(rank, dev):
     return q, kp, vp, bt, cs, lens
 
 
-def decode_bytes(lens, splits):
+def decode_bytes(lens):
     c = DECODE
     kv = sum(lens) * c["Hkv"] * c["d"] * 2 * 2               # K and V, valid tokens only
     io = c["B"] * c["Sq"] * c["H"] * c["d"] * 2 * 2          # q in, out
     io += c["B"] * c["H"] * c["Sq"] * 4                       # lse
     bt = sum((L + c["page"] - 1) // c["page"] for L in lens) * 4 + c["B"] * 4
     return kv + io + bt
+
+
+def _stats(ms_list):
+    """Per-launch times (ms) of one kernel over the timed steps."""
+    return {"median_ms": round(statistics.median(ms_list), 5), "min_ms": round(min(ms_list), 5),
+            "mean_ms": round(sum(ms_list) / len(ms_list), 5), "launch_samples": len(ms_list)}
 
 
 def run_ours(args, rank, world, local):
@@ -214,10 +232,13 @@ def run_ours(args, rank, world, local):
         DECODE.update(B=2, lo=1024, hi=1024)
     dq, kp, vp, bt, cs, lens = make_decode(rank, dev)
     dq_d, bt_d, cs_d = dq.to(dev), bt.to(dev), cs.to(dev)
-    splits = args.num_splits
+    # the headline split count first, then the others of the workload; 1 is the
+    # unsplit control (one CTA per (sequence, KV head): imbalanced by design)
+    split_list = [args.num_splits] + [x for x in (16, 4, 1) if x != args.num_splits]
     c = DECODE
-    ws_bytes = fa.fa_kvcache_workspace_size(c["B"], c["Sq"], c["H"], c["Hkv"], c["d"],
-                                            bt.shape[1] * c["page"], c["page"], splits)
+    ws_bytes = max(fa.fa_kvcache_workspace_size(c["B"], c["Sq"], c["H"], c["Hkv"], c["d"],
+                                                bt.shape[1] * c["page"], c["page"], x)
+                   for x in split_list)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     out_d = torch.empty_like(dq_d)
     lse_d = torch.empty((c["B"], c["H"], c["Sq"]), dtype=torch.float32, device=dev)
@@ -226,98 +247,128 @@ def run_ours(args, rank, world, local):
 
     do_pre = args.only in ("all", "prefill")
     do_dec = args.only in ("all", "decode")
+    R = max(1, args.repeat)
 
     def prefill():
-        if do_pre:
-            fa.fa_fwd(qd_, kd_, vd_, out=out_p, lse=lse_p, causal=True, stream=stream)
+        fa.fa_fwd(qd_, kd_, vd_, out=out_p, lse=lse_p, causal=True, stream=stream)
 
-    def decode():
-        if do_dec:
-            fa.fa_fwd_kvcache(dq_d, kp, vp, cache_seqlens=cs_d, block_table=bt_d, causal=True,
-                              num_splits=splits, out=out_d, lse=lse_d, workspace=ws,
-                              stream=stream)
+    def decode(splits, o=None, l=None):
+        fa.fa_fwd_kvcache(dq_d, kp, vp, cache_seqlens=cs_d, block_table=bt_d, causal=True,
+                          num_splits=splits, out=out_d if o is None else o,
+                          lse=lse_d if l is None else l, workspace=ws, stream=stream)
 
+    groups = ([("prefill", prefill)] if do_pre else []) + (
+        [(f"decode_s{x}", (lambda x=x: decode(x))) for x in split_list] if do_dec else [])
     for _ in range(args.warmup):
         flush.zero_()
-        prefill()
-        decode()
+        for _, fn in groups:
+            fn()
     torch.cuda.synchronize(dev)
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(groups) + 1)] for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize(dev)
     with Clocks(dev.index if dev.index is not None else 0) as clk:
         for s in range(K):
             flush.zero_()                       # L2 flushed between steps (not timed)
             ev[s][0].record(stream)
-            prefill()
-            ev[s][1].record(stream)
-            decode()
-            ev[s][2].record(stream)
+            for g, (_, fn) in enumerate(groups):
+                for _ in range(R):              # inputs exceed L2: back-to-back launches
+                    fn()
+                ev[s][g + 1].record(stream)
         torch.cuda.synchronize(dev)
     barrier(world)
-    t_pre = sum(e[0].elapsed_time(e[1]) for e in ev) / K      # ms per launch
-    t_dec = sum(e[1].elapsed_time(e[2]) for e in ev) / K
-    t_pre = max(t_pre, 1e-9)
-    t_dec = max(t_dec, 1e-9)
-    t_step = t_pre + t_dec
-    t_pre_max = max_over_ranks(t_pre, world)
-    t_dec_max = max_over_ranks(t_dec, world)
+    per = {name: [ev[s][g].elapsed_time(ev[s][g + 1]) / R for s in range(K)]
+           for g, (name, _) in enumerate(groups)}
+    st = {name: _stats(v) for name, v in per.items()}
+    t_step = statistics.median(ev[s][0].elapsed_time(ev[s][-1]) for s in range(K))
     t_step_max = max_over_ranks(t_step, world)
     assert fa.fa_device_status(clear=True) == 0, "device status flags raised during the bench"
 
     flops = prefill_flops()
-    tflops = flops / (t_pre_max * 1e-3) / 1e12 * world
-    dbytes = decode_bytes(lens, splits)
-    gbs = dbytes / (t_dec_max * 1e-3) / 1e9 * world
+    dbytes = decode_bytes(lens)
     res = {
-        "metric": METRIC,
-        "value": round(tflops, 2),
-        "unit": "TFLOPS",
-        "n_gpus": world,
-        "steps": K,
-        "warmup": args.warmup,
-        "ms_per_step": round(t_step_max, 4),
-        "higher_is_better": True,
-        "scaling": "weak",
+        "metric": METRIC, "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(t_step_max, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
         "dtype": "fp16 (prefill), bf16 (decode); fp32 accumulate",
         "data": "synthetic (seeded N(0,1))",
         "config": {
             "workload": (f"causal prefill B={PREFILL['B']} S={PREFILL['S']} H={PREFILL['H']} "
                          f"d={PREFILL['d']} {PREFILL['dtype']} + paged split-KV decode "
-                         f"B={DECODE['B']} H=32 Hkv=8 d=128 bf16 cache U{{1K..32K}} page 256"),
-            "prefill": dict(PREFILL, ms=round(t_pre_max, 4), flop=flops),
-            "decode": dict(DECODE, num_splits=splits, sum_cache_tokens=int(sum(lens)),
-                           ms=round(t_dec_max, 4), bytes=dbytes),
-            "l2": "flushed between steps (256 MiB write, untimed)",
+                         f"B={DECODE['B']} H=32 Hkv=8 d=128 bf16 cache U{{1K..32K}} page 256 "
+                         f"at num_splits {split_list}"),
+            "prefill": dict(PREFILL, flop=flops),
+            "decode": dict(DECODE, num_splits=split_list, sum_cache_tokens=int(sum(lens)),
+                           bytes=dbytes),
+            "launches_per_kernel_per_step": R,
+            "l2": ("flushed between steps (256 MiB write, untimed); within a step each kernel "
+                   "runs back to back on inputs larger than L2 (prefill q/k/v "
+                   f"{3 * q.numel() * q.element_size() >> 20} MiB, decode KV cache "
+                   f"{(kp.numel() + vp.numel()) * kp.element_size() >> 20} MiB)"),
             "parallelism": f"dp{world} (independent replicas)",
         },
-        "decode": {
-            "value": round(gbs, 1), "unit": "GB/s", "ms": round(t_dec_max, 4),
-            "roofline": {"bound": "hbm", "achieved": round(dbytes / (t_dec_max * 1e-3) / 1e9, 1),
-                         "peak": hbm_peak, "unit": "GB/s",
-                         "frac": round(dbytes / (t_dec_max * 1e-3) / 1e9 / hbm_peak, 4),
-                         "traffic": (profiled_traffic("decode_kernel_paged_B8.md",
-                                                      ["decode_kernel.cuh", "decode.cu",
-                                                       "sm100.cuh", "fa_internal.h"])
-                                     if (DECODE["B"] == 64 and splits == 16) else None),
-                         "peak_source": peak_src},
-        },
-        "roofline": {"bound": "tensor", "achieved": round(flops / (t_pre * 1e-3) / 1e12, 2),
-                     "peak": tflops_peak, "unit": "TFLOP/s",
-                     "frac": round(flops / (t_pre * 1e-3) / 1e12 / tflops_peak, 4),
-                     "traffic": (profiled_traffic("fwd_kernel_d64_causal_B4_S4096.md",
-                                                  ["fwd_kernel.cuh", "fwd_launch.cuh",
-                                                   "sm100.cuh", "fa_internal.h"])
-                                 if (PREFILL["d"] == 64 and PREFILL["S"] == 4096) else None),
-                     "kernel": f"fwd_kernel<{PREFILL['d']}, {PREFILL['dtype']}, causal>",
-                     "peak_source": f"{peak_src} bf16 burst (fp16 dense rate equals bf16)"},
-        "gpu_launches": K * ((1 if do_pre else 0) + ((2 if splits > 1 else 1) if do_dec else 0)),
+        # per decode call: the prep kernel (counter, longest-first order), the split
+        # kernel and, above one split, the combine kernel
+        "gpu_launches": K * R * ((1 if do_pre else 0) +
+                                 (sum(3 if x > 1 else 2 for x in split_list) if do_dec else 0)),
         "clocks": clk.summary(),
     }
-    if not args.no_e2e:
-        res["e2e"] = e2e_prefill(fa, q, k, v, dev, stream, flops, world)
+    if do_pre:
+        t_pre = max_over_ranks(st["prefill"]["median_ms"], world)
+        achieved = flops / (st["prefill"]["median_ms"] * 1e-3) / 1e12
+        res["value"] = round(flops / (t_pre * 1e-3) / 1e12 * world, 2)
+        res["prefill"] = dict(st["prefill"], tflops_median=round(achieved, 2),
+                              tflops_best=round(flops / (st["prefill"]["min_ms"] * 1e-3) / 1e12, 2))
+        res["roofline"] = {
+            "bound": "tensor", "achieved": round(achieved, 2), "peak": tflops_peak,
+            "unit": "TFLOP/s", "frac": round(achieved / tflops_peak, 4),
+            "traffic": (profiled_traffic("fwd_kernel_d64_causal_B4_S4096.md",
+                                         ["fwd_kernel.cuh", "fwd_launch.cuh", "sm100.cuh",
+                                          "fa_internal.h"])
+                        if (PREFILL["d"] == 64 and PREFILL["S"] == 4096) else None),
+            "kernel": f"fwd_kernel<{PREFILL['d']}, {PREFILL['dtype']}, causal>",
+            "peak_source": f"{peak_src} bf16 burst (fp16 dense rate equals bf16)"}
+        sus = sustained_tflops()
+        if sus:
+            # the step repeats each kernel back to back for about a second, which can bring
+            # the power cap in (see clocks); the GEMM rate measured under it, for context
+            res["roofline"]["frac_vs_sustained_peak"] = round(achieved / sus, 4)
+            res["roofline"]["sustained_peak"] = sus
+    if do_dec:
+        by = {}
+        for x in split_list:
+            sx = st[f"decode_s{x}"]
+            gbs = dbytes / (sx["median_ms"] * 1e-3) / 1e9
+            by[str(x)] = dict(sx, gbs_median=round(gbs, 1),
+                              gbs_best=round(dbytes / (sx["min_ms"] * 1e-3) / 1e9, 1),
+                              frac=round(gbs / hbm_peak, 4),
+                              role=("headline" if x == args.num_splits else
+                                    "unsplit control" if x == 1 else "reported"))
+        main = by[str(args.num_splits)]
+        t_dec = max_over_ranks(main["median_ms"], world)
+        res["decode"] = {
+            "value": round(dbytes / (t_dec * 1e-3) / 1e9 * world, 1), "unit": "GB/s",
+            "num_splits": args.num_splits, "ms": round(t_dec, 5),
+            "roofline": {"bound": "hbm", "achieved": main["gbs_median"], "peak": hbm_peak,
+                         "unit": "GB/s", "frac": main["frac"],
+                         "traffic": (profiled_traffic(f"decode_kernel_paged_B64_s{args.num_splits}.md",
+                                                      ["decode_kernel.cuh", "decode.cu",
+                                                       "sm100.cuh", "fa_internal.h"])
+                                     if DECODE["B"] == 64 else None),
+                         "kernel": "decode_kernel<128, bf16> + combine_kernel",
+                         "peak_source": peak_src},
+            "by_num_splits": by}
+        if not do_pre:
+            res.update(value=res["decode"]["value"], unit="GB/s")
+    if not args.no_e2e and do_pre:
+        res["e2e"] = e2e_prefill(fa, q, k, v, dev, stream, flops, world, steps=K)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(args, gpu=dict(
+            q=q, k=k, v=v, out=out_p if do_pre else None, lse=lse_p if do_pre else None,
+            dq=dq, kp=kp, vp=vp, bt=bt, cs=cs, lens=lens,
+            decode=(lambda x, o, l: decode(x, o, l)) if do_dec else None, splits=split_list,
+            dev=dev, stream=stream))
     return res
 
 
@@ -404,7 +455,9 @@ SWEEP = dict(B=4, H=32, d=(64, 128), S=(512, 1024, 2048, 4096, 8192, 16384),
 def run_sweep(args, rank, world, local):
     """--only sweep: the causal prefill's TFLOPS over head dims, sequence lengths
     and 16-bit types; one JSON line whose value is the largest point (d=128,
-    S=16384, bf16) and whose ``curve`` holds every point."""
+    S=16384, bf16) and whose ``curve`` holds every point with its own clock record
+    (each point launches for at least ~0.3 s, L2 flushed between launches, so the
+    100 ms sampler sees it)."""
     import io_aware_online_b200 as fa
     from io_aware_online_b200 import build as fa_build
     fa_build.build()
@@ -414,44 +467,61 @@ def run_sweep(args, rank, world, local):
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     c = SWEEP
-    K = min(args.steps, 10)
     curve = []
-    with Clocks(dev.index if dev.index is not None else 0) as clk:
-        for d in c["d"]:
-            for S in c["S"]:
-                for dname in c["dtype"]:
-                    dt = synth.DTYPES[dname]
-                    gen = torch.Generator(device=dev).manual_seed(3300 + S + d + rank)
-                    shp = (c["B"], S, c["H"], d)
-                    q, k, v = (torch.randn(shp, generator=gen, device=dev).to(dt)
-                               for _ in range(3))
-                    out = torch.empty_like(q)
-                    lse = torch.empty((c["B"], c["H"], S), dtype=torch.float32, device=dev)
-                    for _ in range(args.warmup):
-                        flush.zero_()
-                        fa.fa_fwd(q, k, v, out=out, lse=lse, causal=True, stream=stream)
-                    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
-                          for _ in range(K)]
-                    barrier(world)
-                    torch.cuda.synchronize(dev)
+    launches = 0
+    all_reasons = set()
+    for d in c["d"]:
+        for S in c["S"]:
+            for dname in c["dtype"]:
+                dt = synth.DTYPES[dname]
+                gen = torch.Generator(device=dev).manual_seed(3300 + S + d + rank)
+                shp = (c["B"], S, c["H"], d)
+                q, k, v = (torch.randn(shp, generator=gen, device=dev).to(dt) for _ in range(3))
+                out = torch.empty_like(q)
+                lse = torch.empty((c["B"], c["H"], S), dtype=torch.float32, device=dev)
+
+                def call():
+                    fa.fa_fwd(q, k, v, out=out, lse=lse, causal=True, stream=stream)
+                for _ in range(args.warmup):
+                    flush.zero_()
+                    call()
+                torch.cuda.synchronize(dev)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                call()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                est = max(e0.elapsed_time(e1), 1e-3)
+                K = max(min(args.steps, 10), int(300.0 / (est + 0.05)) + 1)
+                ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+                barrier(world)
+                torch.cuda.synchronize(dev)
+                with Clocks(dev.index if dev.index is not None else 0) as clk:
                     for i in range(K):
                         flush.zero_()
                         ev[i][0].record(stream)
-                        fa.fa_fwd(q, k, v, out=out, lse=lse, causal=True, stream=stream)
+                        call()
                         ev[i][1].record(stream)
                     torch.cuda.synchronize(dev)
-                    barrier(world)
-                    ms = max_over_ranks(statistics.median(e[0].elapsed_time(e[1]) for e in ev),
-                                        world)
-                    tf = 4.0 * d * c["B"] * c["H"] * causal_pairs(S, S) / (ms * 1e-3) / 1e12
-                    curve.append({"d": d, "S": S, "dtype": dname, "ms": round(ms, 4),
-                                  "tflops": round(tf, 1), "frac": round(tf / tflops_peak, 4)})
-                    del q, k, v, out, lse
+                barrier(world)
+                launches += K
+                ms = max_over_ranks(statistics.median(e[0].elapsed_time(e[1]) for e in ev),
+                                    world)
+                ms_min = min(e[0].elapsed_time(e[1]) for e in ev)
+                flop = 4.0 * d * c["B"] * c["H"] * causal_pairs(S, S)
+                tf = flop / (ms * 1e-3) / 1e12
+                ck = clk.summary()
+                all_reasons.update(ck.get("reasons", []))
+                curve.append({"d": d, "S": S, "dtype": dname, "ms": round(ms, 4),
+                              "tflops": round(tf, 1),
+                              "tflops_best": round(flop / (ms_min * 1e-3) / 1e12, 1),
+                              "frac": round(tf / tflops_peak, 4), "launches": K, "clocks": ck})
+                del q, k, v, out, lse
     assert fa.fa_device_status(clear=True) == 0, "device status flags raised during the sweep"
     top = curve[-1]
     return {"metric": "attn fwd TFLOPS vs seqlen (causal prefill)",
             "value": round(top["tflops"] * world, 2), "unit": "TFLOPS", "n_gpus": world,
-            "steps": K, "warmup": args.warmup, "ms_per_step": top["ms"],
+            "steps": top["launches"], "warmup": args.warmup, "ms_per_step": top["ms"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp16 / bf16; fp32 accumulate", "data": "synthetic (seeded N(0,1))",
             "config": {"workload": "causal prefill sweep B=4 H=32 over d, S and dtype; value = "
@@ -461,7 +531,8 @@ def run_sweep(args, rank, world, local):
             "roofline": {"bound": "tensor", "achieved": top["tflops"], "peak": tflops_peak,
                          "unit": "TFLOP/s", "frac": top["frac"], "traffic": None,
                          "kernel": "fwd_kernel<128, bf16, causal>", "peak_source": peak_src},
-            "curve": curve, "gpu_launches": K * len(curve), "clocks": clk.summary()}
+            "curve": curve, "gpu_launches": launches,
+            "clocks": {"per_point": True, "reasons": sorted(all_reasons)}}
 
 
 def run_fp8(args, rank, world, local):
@@ -647,25 +718,105 @@ def oracle_prefill_sample(heads: int, threads: int):
     return flops / dt / 1e12, dt
 
 
-def cpu_baseline(args):
-    # up to all 128 (b, h) problems of the workload, eight per host core (about 10 s on
-    # a 16-core host); the problems are independent, so the rate is the workload's
+def _max_abs(a, b):
+    import numpy as np
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    fin = np.isfinite(b)
+    if not np.array_equal(np.isfinite(a), fin) or not np.array_equal(a[~fin], b[~fin]):
+        return float("inf")
+    return float(np.abs(a[fin] - b[fin]).max()) if fin.any() else 0.0
+
+
+def cpu_baseline(args, gpu=None):
+    """The fp64 oracle on the host cores: timed on a bounded sample of the prefill
+    workload's own (b, h) problems (eight per core, about 10 s on 16 cores), whose
+    outputs also give the sample's max |dO| and |dLSE| against the GPU run; plus
+    single-thread times of the two small parity configurations."""
+    import numpy as np
+
+    import oracle
     cores = max(1, os.cpu_count() or 1)
-    problems = min(PREFILL["B"] * PREFILL["H"], 8 * cores)
-    tf, dt = oracle_prefill_sample(problems, cores)
-    return {"value": round(tf, 6), "unit": "TFLOPS", "cores": cores, "kind": "oracle",
-            "sample": f"prefill workload, {problems} of its {PREFILL['B'] * PREFILL['H']} "
-                      f"(b, h) problems, full S={PREFILL['S']} causal (fp64 C oracle, "
-                      f"OpenMP over problems), {dt:.1f} s"}
+    c = PREFILL
+    res = {"unit": "TFLOPS", "cores": cores, "kind": "oracle"}
+    if gpu is not None and gpu["out"] is not None:
+        q, k, v = gpu["q"], gpu["k"], gpu["v"]
+        problems = min(c["B"] * c["H"], 8 * cores)
+        nb = (problems + c["H"] - 1) // c["H"]
+        ro_all, rl_all = [], []
+        t0 = time.perf_counter()
+        for b in range(nb):
+            nh = min(c["H"], problems - b * c["H"])
+            ro, rl = oracle.attention_dense(q[b:b + 1, :, :nh], k[b:b + 1, :, :nh],
+                                            v[b:b + 1, :, :nh], causal=True, threads=cores)
+            ro_all.append((b, nh, ro))
+            rl_all.append((b, nh, rl))
+        dt = time.perf_counter() - t0
+        flops = 4.0 * c["d"] * problems * causal_pairs(c["S"], c["S"])
+        go = gpu["out"].float().cpu().numpy()
+        gl = gpu["lse"].cpu().numpy()
+        d_o = max(_max_abs(go[b:b + 1, :, :nh], ro) for b, nh, ro in ro_all)
+        d_l = max(_max_abs(gl[b:b + 1, :nh], rl) for b, nh, rl in rl_all)
+        res.update(value=round(flops / dt / 1e12, 6),
+                   sample=(f"prefill workload, its first {problems} of {c['B'] * c['H']} (b, h) "
+                           f"problems, full S={c['S']} causal (fp64 C oracle, OpenMP over "
+                           f"problems, {cores} threads), {dt:.1f} s"),
+                   parity={"prefill": {"max_abs_dO": d_o, "max_abs_dLSE": d_l,
+                                       "problems": problems,
+                                       "tolerance": {"dO": 2e-3 if c["dtype"] == "fp16" else 1e-2,
+                                                     "dLSE": 1e-3}}})
+    else:
+        problems = min(c["B"] * c["H"], 8 * cores)
+        tf, dt = oracle_prefill_sample(problems, cores)
+        res.update(value=round(tf, 6),
+                   sample=f"{problems} (b, h) problems of S={c['S']} causal, {dt:.1f} s")
+    if gpu is not None and gpu["decode"] is not None:
+        # the first eight sequences of the decode batch, every head, at each split count
+        n = min(8, len(gpu["lens"]))
+        dev, D = gpu["dev"], DECODE
+        # only their pages reach the host: a compact pool and a remapped block table
+        bt_n = gpu["bt"][:n].clone()
+        ids = sorted({int(x) for x in bt_n.flatten().tolist() if x >= 0})
+        remap = {b: i for i, b in enumerate(ids)}
+        bt_c = bt_n.apply_(lambda x: remap[x] if x >= 0 else -1)
+        idx = torch.tensor(ids, dtype=torch.long, device=gpu["kp"].device)
+        kc = gpu["kp"].index_select(0, idx).cpu()
+        vc = gpu["vp"].index_select(0, idx).cpu()
+        ro, rl = oracle.attention_paged(gpu["dq"][:n], kc, vc, bt_c, gpu["cs"][:n], causal=True,
+                                        threads=cores)
+        par = {}
+        for x in gpu["splits"]:
+            o = torch.empty((D["B"], D["Sq"], D["H"], D["d"]), dtype=torch.bfloat16, device=dev)
+            lz = torch.empty((D["B"], D["H"], D["Sq"]), dtype=torch.float32, device=dev)
+            gpu["decode"](x, o, lz)
+            torch.cuda.synchronize(dev)
+            par[str(x)] = {"max_abs_dO": _max_abs(o[:n].float().cpu().numpy(), ro),
+                           "max_abs_dLSE": _max_abs(lz[:n].cpu().numpy(), rl)}
+        res.setdefault("parity", {})["decode"] = dict(
+            by_num_splits=par, sequences=n, tolerance={"dO": 1e-2, "dLSE": 1e-3})
+    # single-thread oracle times of the tiny and the causal Sq != Sk configurations
+    one = {}
+    for name, (B, Sq, Sk, H, d, dt_, causal) in {
+            "tiny B1 H2 S128 d64 fp16": (1, 128, 128, 2, 64, torch.float16, False),
+            "causal B2 H8 Sq384 Sk1024 d128 bf16": (2, 384, 1024, 8, 128, torch.bfloat16, True)
+    }.items():
+        qq, kk, vv = synth.dense(B, Sq, Sk, H, H, d, dt_, seed=1001)
+        t0 = time.perf_counter()
+        oracle.attention_dense(qq, kk, vv, causal=causal, threads=1)
+        one[name] = round((time.perf_counter() - t0) * 1e3, 3)
+    res["single_thread_ms"] = one
+    return res
 
 
 def run_reference(args, rank, world):
-    """The reference arm: the fp64 CPU oracle on bounded samples of the prefill workload."""
-    heads = max(1, min(8, os.cpu_count() or 1))        # one OpenMP thread per head
-    cores = heads
+    """The reference arm: the fp64 CPU oracle, on all host cores (one OpenMP thread per
+    (b, h) problem, as many problems per step as cores), on bounded samples of the
+    prefill workload."""
+    cores = max(1, os.cpu_count() or 1)
+    heads = max(1, min(PREFILL["B"] * PREFILL["H"], cores))
     times = []
     for i in range(args.warmup + args.steps):
-        tf, dt = oracle_prefill_sample(heads, heads)
+        tf, dt = oracle_prefill_sample(heads, cores)
         if i >= args.warmup:
             times.append((tf, dt))
     tf = statistics.median(t for t, _ in times)
@@ -675,10 +826,11 @@ def run_reference(args, rank, world):
             "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
             "config": {"workload": "causal prefill B=4 S=4096 H=32 d=64 (bounded sample: "
-                                   f"batch 0, {heads} heads per step)"},
+                                   f"{heads} (b, h) problems per step)"},
             "cpu_baseline": {"value": round(tf, 6), "unit": "TFLOPS", "cores": cores,
                              "kind": "oracle",
-                             "sample": f"{heads} heads x full S=4096 causal per step"},
+                             "sample": f"{heads} heads x full S=4096 causal per step, "
+                                       f"{cores} threads"},
             "e2e": {"value": round(tf, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -689,7 +841,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--num-splits", type=int, default=16)
+    ap.add_argument("--num-splits", type=int, default=4,
+                    help="the decode's headline split count (16 and 1 are timed beside it)")
+    ap.add_argument("--repeat", type=int, default=10,
+                    help="back-to-back launches of each kernel per step (inputs exceed L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "chunked", "append", "fp8",
@@ -721,8 +876,6 @@ def main():
             return
         res = run_ours(args, rank, world, local)
         if rank == 0:
-            if not args.no_cpu_baseline and world == 1:
-                res["cpu_baseline"] = cpu_baseline(args)
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:

@@ -185,10 +185,11 @@ FA_API size_t fa_kvcache_workspace_size(int batch, int seqlen_q, int num_heads, 
  *   second kernel combines them (fa_combine's arithmetic).  The result does not
  *   depend on num_splits beyond rounding.
  * workspace: device scratch of at least fa_kvcache_workspace_size(...) bytes,
- *   16-byte aligned, required.  It holds the split kernel's work-item counter
- *   (zeroed by the call with an asynchronous memset on `stream`) and the fp32
- *   split partials between the two kernels of one call, so calls that share a
- *   workspace must be stream-ordered.
+ *   16-byte aligned, required.  It holds the split kernel's work-item counter and
+ *   the longest-first order of the sequences (both written by a small kernel the
+ *   call launches on `stream` first; the split kernel claims the items of the
+ *   longest sequences first) and the fp32 split partials between the kernels of one
+ *   call, so calls that share a workspace must be stream-ordered.
  * Up to 16 query rows per KV head ((num_heads / num_heads_k) * seqlen_q) the call
  *   runs the split-KV decode kernel above.  With more (chunked prefill against the
  *   cache: a chunk of new query rows attends everything cached, causal aligned
@@ -261,31 +262,41 @@ FA_API int fa_fwd_kvcache_append(const void *q, void *k_cache, void *v_cache, co
 FA_API size_t fa_bwd_workspace_size(int batch, int seqlen_q, int num_heads);
 
 /*
- * fa_bwd -- gradients of the dense attention forward (tag page "flash attention":
- * the backward recomputes the attention matrix tile by tile from Q, K and the
+ * fa_bwd -- gradients of the attention forward (tag page "flash attention": the
+ * backward recomputes the attention matrix tile by tile from Q, K and the
  * forward's softmax statistics instead of reading a stored one).
  *
+ * Dense (cu_seqlens_q == cu_seqlens_k == NULL):
  *   dout, q, out, dq: [batch, seqlen_q, num_heads, head_dim] contiguous, 16-bit
  *   (dtype as for fa_fwd); k, v, dk, dv: [batch, seqlen_k, num_heads_k, head_dim]
- *   contiguous; lse: fp32 [batch, num_heads, seqlen_q], the forward's LSE;
- *   out: the forward's O.  The mask, scale, window and ALiBi arguments must be
- *   those of the forward call; softcap must be 0 (its backward is not built:
- *   FA_ERR_UNSUPPORTED).
- * Computes, with P = exp(scale Q K^T + bias - LSE) on the allowed entries and
- * D = rowsum(dout * out): dv = P^T dout, dS = P * (dout v^T - D),
- * dq = scale dS k, dk = scale dS^T q; dk and dv sum over the query heads that
+ *   contiguous; lse: fp32 [batch, num_heads, seqlen_q], the forward's LSE.
+ * Varlen (both cu_seqlens non-NULL, device int32 [batch + 1] as for fa_fwd,
+ *   section 3.2): the same tensors packed along the rows, [total_q, num_heads,
+ *   head_dim] and [total_k, num_heads_k, head_dim] with seqlen_q / seqlen_k the
+ *   packed totals; lse fp32 [num_heads, total_q] (fa_fwd's varlen layout);
+ *   max_seqlen_q / max_seqlen_k bound every sequence's lengths.  Each sequence
+ *   is its own problem, its mask aligned bottom-right within it.
+ * out: the forward's O.  The mask, scale, window, softcap and ALiBi arguments
+ * must be those of the forward call.
+ * Computes, with X = scale Q K^T, T = tanh(X / softcap) and S = softcap T
+ * (S = X without a softcap; changelog v2.6, section 5.2), P = exp(S + bias - LSE)
+ * on the allowed entries and D = rowsum(dout * out): dv = P^T dout,
+ * dS = P * (dout v^T - D), dX = dS * (1 - T^2) (dX = dS without a softcap),
+ * dq = scale dX k, dk = scale dX^T q; dk and dv sum over the query heads that
  * share a KV head.  Deterministic (no atomics): one pass per key block for dk/dv,
- * one per query block for dq.  P and dS are rounded to the input dtype before
+ * one per query block for dq.  P and dX are rounded to the input dtype before
  * their products (fp32 accumulation).
- * workspace: >= fa_bwd_workspace_size(batch, seqlen_q, num_heads) bytes, 16-byte
- *   aligned; calls sharing it must be stream-ordered.
+ * workspace: >= fa_bwd_workspace_size(batch, seqlen_q, num_heads) bytes (varlen:
+ *   fa_bwd_workspace_size(1, total_q, num_heads)), 16-byte aligned; calls sharing
+ *   it must be stream-ordered.
  */
 FA_API int fa_bwd(const void *dout, const void *q, const void *k, const void *v,
                   const void *out, const float *lse, void *dq, void *dk, void *dv, int dtype,
                   int batch, int seqlen_q, int seqlen_k, int num_heads, int num_heads_k,
-                  int head_dim, float softmax_scale, int causal, int window_left,
-                  int window_right, float softcap, const float *alibi_slopes, void *workspace,
-                  size_t workspace_bytes, void *stream);
+                  int head_dim, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                  int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal,
+                  int window_left, int window_right, float softcap, const float *alibi_slopes,
+                  void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * fa_selftest_wait_timeout -- a diagnostic of the bounded waits (the pages have no

@@ -94,7 +94,7 @@ def load():
     lib.fa_bwd_workspace_size.argtypes = [i32, i32, i32]
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
-                           f32, i32, i32, i32, f32, vp, vp, ctypes.c_size_t, vp]
+                           vp, vp, i32, i32, f32, i32, i32, i32, f32, vp, vp, ctypes.c_size_t, vp]
     lib.fa_bwd.restype = i32
     lib.fa_selftest_wait_timeout.argtypes = [i32, vp]
     lib.fa_selftest_wait_timeout.restype = i32
@@ -368,27 +368,46 @@ def fa_selftest_wait_timeout(timeout_ms=20, stream=None):
     _check(load().fa_selftest_wait_timeout(int(timeout_ms), _stream(stream)))
 
 
-def fa_bwd(dout, q, k, v, out, lse, *, softmax_scale=None, causal=False, window_size=(-1, -1),
-           alibi_slopes=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """Gradients (dq, dk, dv) of the dense forward for output gradient dout; q, out,
-    dout [B, Sq, H, d], k, v [B, Sk, Hkv, d] contiguous, lse [B, H, Sq] from fa_fwd
-    (same mask arguments as the forward call)."""
+def fa_bwd(dout, q, k, v, out, lse, *, cu_seqlens_q=None, cu_seqlens_k=None,
+           max_seqlen_q=None, max_seqlen_k=None, softmax_scale=None, causal=False,
+           window_size=(-1, -1), softcap=0.0, alibi_slopes=None, dq=None, dk=None, dv=None,
+           workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of the forward for output gradient dout (same mask,
+    scale, softcap and ALiBi arguments as the forward call).
+    Dense: q, out, dout [B, Sq, H, d], k, v [B, Sk, Hkv, d] contiguous, lse [B, H, Sq].
+    Varlen: q, out, dout [total_q, H, d], k, v [total_k, Hkv, d], int32 cu_seqlens
+    [B+1], max_seqlen_q/k, lse [H, total_q] (fa_fwd's varlen outputs)."""
     lib = load()
     dt = _dtype(q)
-    B, sq, H, d = q.shape
-    sk, Hkv = k.shape[1], k.shape[2]
+    varlen = cu_seqlens_q is not None or cu_seqlens_k is not None
+    if varlen:
+        if cu_seqlens_q is None or cu_seqlens_k is None:
+            raise ValueError("varlen needs cu_seqlens_q and cu_seqlens_k")
+        if max_seqlen_q is None or max_seqlen_k is None:
+            raise ValueError("varlen needs max_seqlen_q and max_seqlen_k")
+        B = cu_seqlens_q.numel() - 1
+        sq, H, d = q.shape
+        sk, Hkv = k.shape[0], k.shape[1]
+        ws_b = 1
+    else:
+        B, sq, H, d = q.shape
+        sk, Hkv = k.shape[1], k.shape[2]
+        max_seqlen_q = max_seqlen_k = 0
+        ws_b = B
     for t in (dout, q, k, v, out, lse):
         if not t.is_contiguous():
             raise ValueError("fa_bwd takes contiguous tensors")
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    need = lib.fa_bwd_workspace_size(B, sq, H)
+    need = lib.fa_bwd_workspace_size(ws_b, sq, H)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib.fa_bwd(_ptr(dout), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dq),
-                      _ptr(dk), _ptr(dv), dt, B, sq, sk, H, Hkv, d, _scale(softmax_scale),
-                      int(bool(causal)), int(window_size[0]), int(window_size[1]), 0.0,
-                      _ptr(alibi_slopes), _ptr(workspace), ws_bytes, _stream(stream)))
+                      _ptr(dk), _ptr(dv), dt, B, sq, sk, H, Hkv, d, _ptr(cu_seqlens_q),
+                      _ptr(cu_seqlens_k), int(max_seqlen_q), int(max_seqlen_k),
+                      _scale(softmax_scale), int(bool(causal)), int(window_size[0]),
+                      int(window_size[1]), float(softcap), _ptr(alibi_slopes), _ptr(workspace),
+                      ws_bytes, _stream(stream)))
     return dq, dk, dv

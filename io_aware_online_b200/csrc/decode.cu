@@ -24,6 +24,11 @@ static cudaError_t launch_decode_inst(const CUtensorMap& tk, const CUtensorMap& 
   return cudaGetLastError();
 }
 
+cudaError_t launch_decode_prep(const DecodeParams& p, cudaStream_t stream) {
+  decode_prep_kernel<<<1, 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           bool bf16, int d, cudaStream_t stream) {
   const int rmax = (p.R <= 4) ? 4 : 16;

@@ -14,6 +14,10 @@
 // time from a counter (atomicAdd; items differ in length by up to 32x, so a static
 // assignment leaves a long tail), and within a CTA the stream of 64-token K/V
 // tiles runs on across item boundaries, so no CTA drains its copy pipeline.
+// Items are claimed longest sequence first (a prep kernel ranks the sequences by
+// cache length before the launch), so the last items to finish are the shortest:
+// at 4 splits an item of a 32K-token sequence is 8K tokens, and claimed last it
+// would leave most CTAs idle for its whole duration.
 //   warps 0-3  consumers: warp w owns tokens [16w, 16w+16) of every tile and runs
 //              its own online softmax (max, sum) and P*V over them, with no
 //              barrier between warps inside the tile loop; at the end of an item
@@ -105,6 +109,7 @@ __device__ __forceinline__ DecItem dec_item(const DecodeParams& p, int item) {
   it.split = item % p.num_splits;
   it.hk = (item / p.num_splits) % p.Hkv;
   it.b = item / (p.num_splits * p.Hkv);
+  if (p.order != nullptr) it.b = p.order[it.b];  // longest sequences first
   it.L = ((p.cache_seqlens != nullptr) ? p.cache_seqlens[it.b] : p.seqlen_k_max) + p.k_add;
   {
     // a length the cache cannot hold would read past the block table: clamp it
@@ -131,6 +136,24 @@ __device__ __forceinline__ DecItem dec_item(const DecodeParams& p, int item) {
   it.t_lo = kb_lo / kDecTok;
   it.n_tiles = (kb_hi > kb_lo) ? (kb_hi + kDecTok - 1) / kDecTok - it.t_lo : 0;
   return it;
+}
+
+// One CTA: zero the work-item counter; rank the sequences by attended length,
+// longest first (ties by index), into p.order.  O(B^2 / threads) comparisons for
+// B <= kDecOrderMax.
+__global__ void __launch_bounds__(128) decode_prep_kernel(const DecodeParams p) {
+  if (threadIdx.x == 0) *p.item_counter = 0u;
+  if (p.order == nullptr) return;
+  int16_t* order = const_cast<int16_t*>(p.order);
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+    const int lb = p.cache_seqlens[b];
+    int rank = 0;
+    for (int c = 0; c < p.B; ++c) {
+      const int lc = p.cache_seqlens[c];
+      rank += (lc > lb) || (lc == lb && c < b);
+    }
+    order[rank] = static_cast<int16_t>(b);
+  }
 }
 
 template <int D, bool BF16, int RMAX>

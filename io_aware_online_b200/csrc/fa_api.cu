@@ -388,8 +388,9 @@ int fa_kvcache_num_splits(int batch, int seqlen_q, int num_heads, int num_heads_
 }
 
 // Workspace layout: a 256-byte header (word 0: the decode kernel's work-item counter,
-// zeroed at every call) followed, when the split count is above 1, by the fp32
-// partial outputs [splits, B, Sq, H, D] and partial LSEs [splits, B, Sq, H].
+// zeroed at every call; bytes 16 .. 255: the longest-first order of up to 120
+// sequences, int16) followed, when the split count is above 1, by the fp32 partial
+// outputs [splits, B, Sq, H, D] and partial LSEs [splits, B, Sq, H].
 static constexpr size_t kWsHeader = 256;
 
 size_t fa_kvcache_workspace_size(int batch, int seqlen_q, int num_heads, int num_heads_k,
@@ -584,8 +585,13 @@ static int kvcache_impl(const void* q, const void* k_cache, const void* v_cache,
     e = fa::launch_kv_append(*app, s);
     if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache_append append launch");
   }
-  e = cudaMemsetAsync(p.item_counter, 0, sizeof(unsigned int), s);
-  if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache counter reset");
+  // the counter is zeroed and, for batches of up to kDecOrderMax sequences, their
+  // longest-first order written after it (one small kernel before the split kernel)
+  p.order = (cache_seqlens != nullptr && batch <= fa::kDecOrderMax)
+                ? reinterpret_cast<const int16_t*>(static_cast<uint8_t*>(workspace) + 16)
+                : nullptr;
+  e = fa::launch_decode_prep(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache prep launch");
   e = fa::launch_decode(tk, tv, p, dtype == FA_BF16, d, s);
   if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_kvcache split kernel launch");
   if (splits > 1) {
@@ -625,12 +631,13 @@ size_t fa_bwd_workspace_size(int batch, int seqlen_q, int num_heads) {
   return (2 * half + 255) / 256 * 256;
 }
 
-// 2-D fp32 tensor map over [rows, cols] with a row stride in bytes, box {128, 1}.
+// 2-D fp32 tensor map over [rows, cols] with a row stride in bytes, box {box_cols, 1}
+// (box_cols * 4 a multiple of 16 bytes).
 static int encode_vec_rows(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t rows,
-                           uint64_t stride_bytes, const char* what) {
+                           uint64_t stride_bytes, uint32_t box_cols, const char* what) {
   cuuint64_t gd[2] = {cols, rows};
   cuuint64_t gs[1] = {stride_bytes};
-  cuuint32_t bx[2] = {128, 1};
+  cuuint32_t bx[2] = {box_cols, 1};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), gd, gs,
                         bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -641,14 +648,20 @@ static int encode_vec_rows(CUtensorMap* map, const void* ptr, uint64_t cols, uin
 
 int fa_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out,
            const float* lse, void* dq, void* dk, void* dv, int dtype, int batch, int seqlen_q,
-           int seqlen_k, int num_heads, int num_heads_k, int head_dim, float softmax_scale,
-           int causal, int window_left, int window_right, float softcap,
-           const float* alibi_slopes, void* workspace, size_t workspace_bytes, void* stream) {
+           int seqlen_k, int num_heads, int num_heads_k, int head_dim,
+           const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int max_seqlen_q,
+           int max_seqlen_k, float softmax_scale, int causal, int window_left, int window_right,
+           float softcap, const float* alibi_slopes, void* workspace, size_t workspace_bytes,
+           void* stream) {
   g_err.clear();
   int rc = check_common(dtype, head_dim, num_heads, num_heads_k, window_left, window_right, softcap);
   if (rc != FA_OK) return rc;
-  if (softcap > 0.f)
-    return fail(FA_ERR_UNSUPPORTED, "fa_bwd: softcap is not supported by the backward pass");
+  const bool varlen = cu_seqlens_q != nullptr || cu_seqlens_k != nullptr;
+  if (varlen && (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr))
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd: varlen needs both cu_seqlens_q and cu_seqlens_k");
+  if (varlen && (max_seqlen_q < 0 || max_seqlen_k < 0 || max_seqlen_q > seqlen_q ||
+                 max_seqlen_k > seqlen_k))
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd: max_seqlen must lie in [0, total rows]");
   if (!dout || !q || !k || !v || !out || !lse || !dq || !dk || !dv)
     return fail(FA_ERR_INVALID_ARG, "fa_bwd: every tensor argument must be non-NULL");
   if (!aligned16(dout) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
@@ -659,7 +672,9 @@ int fa_bwd(const void* dout, const void* q, const void* k, const void* v, const 
   float scale;
   if ((rc = resolve_scale(softmax_scale, head_dim, &scale)) != FA_OK) return rc;
   const int H = num_heads, Hkv = num_heads_k, d = head_dim;
-  const size_t need = fa_bwd_workspace_size(batch, seqlen_q, H);
+  // tensors, maps and statistics of a varlen call are those of one packed batch entry
+  const int bm = varlen ? 1 : batch;
+  const size_t need = fa_bwd_workspace_size(bm, seqlen_q, H);
   if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
     return fail(FA_ERR_WORKSPACE, "fa_bwd: needs %zu bytes of 16-byte aligned workspace (got %zu)",
                 need, workspace_bytes);
@@ -668,14 +683,16 @@ int fa_bwd(const void* dout, const void* q, const void* k, const void* v, const 
     cudaStream_t s0 = static_cast<cudaStream_t>(stream);
     cudaError_t e0 = cudaSuccess;
     if (seqlen_k > 0) {
-      const size_t kv = static_cast<size_t>(batch) * seqlen_k * Hkv * d * 2;
+      const size_t kv = static_cast<size_t>(bm) * seqlen_k * Hkv * d * 2;
       if ((e0 = cudaMemsetAsync(dk, 0, kv, s0)) == cudaSuccess) e0 = cudaMemsetAsync(dv, 0, kv, s0);
     } else {
-      e0 = cudaMemsetAsync(dq, 0, static_cast<size_t>(batch) * seqlen_q * H * d * 2, s0);
+      e0 = cudaMemsetAsync(dq, 0, static_cast<size_t>(bm) * seqlen_q * H * d * 2, s0);
     }
     return e0 == cudaSuccess ? FA_OK : cuda_fail(e0, "fa_bwd zero fill");
   }
-  if (batch > 65535 || H > 65535 || (seqlen_q + 127) / 128 > 65535 || (seqlen_k + 127) / 128 > 65535)
+  const int rows_q = varlen ? max_seqlen_q : seqlen_q;  // per-sequence extents of the grid
+  const int rows_k = varlen ? max_seqlen_k : seqlen_k;
+  if (batch > 65535 || H > 65535 || (rows_q + 127) / 128 > 65535 || (rows_k + 127) / 128 > 65535)
     return fail(FA_ERR_UNSUPPORTED, "fa_bwd: sizes above the grid limits");
   if ((rc = get_encoder()) != FA_OK) return rc;
   unsigned int* status = nullptr;
@@ -684,7 +701,7 @@ int fa_bwd(const void* dout, const void* q, const void* k, const void* v, const 
   const uint32_t box[4] = {64, 128, 1, 1};
   {
     const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(seqlen_q),
-                              static_cast<uint64_t>(H), static_cast<uint64_t>(batch)};
+                              static_cast<uint64_t>(H), static_cast<uint64_t>(bm)};
     const uint64_t st[3] = {static_cast<uint64_t>(H) * d * 2, static_cast<uint64_t>(d) * 2,
                             static_cast<uint64_t>(seqlen_q) * H * d * 2};
     if ((rc = encode_4d(&tq, q, dims, st, box, "q")) != FA_OK) return rc;
@@ -692,7 +709,7 @@ int fa_bwd(const void* dout, const void* q, const void* k, const void* v, const 
   }
   {
     const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(seqlen_k),
-                              static_cast<uint64_t>(Hkv), static_cast<uint64_t>(batch)};
+                              static_cast<uint64_t>(Hkv), static_cast<uint64_t>(bm)};
     const uint64_t st[3] = {static_cast<uint64_t>(Hkv) * d * 2, static_cast<uint64_t>(d) * 2,
                             static_cast<uint64_t>(seqlen_k) * Hkv * d * 2};
     if ((rc = encode_4d(&tk, k, dims, st, box, "k")) != FA_OK) return rc;
@@ -700,13 +717,17 @@ int fa_bwd(const void* dout, const void* q, const void* k, const void* v, const 
   }
   const int sq_pad = (seqlen_q + 3) / 4 * 4;
   float* dvec = static_cast<float*>(workspace);
-  float* lse2 = dvec + static_cast<size_t>(batch) * H * sq_pad;
-  CUtensorMap tl, td;  // rows: the true length, so columns past the end load as 0
-  if ((rc = encode_vec_rows(&tl, lse2, seqlen_q, static_cast<uint64_t>(batch) * H,
-                            static_cast<uint64_t>(sq_pad) * 4, "lse workspace")) != FA_OK)
+  float* lse2 = dvec + static_cast<size_t>(bm) * H * sq_pad;
+  // rows: the true length, so columns past the end load as 0.  Varlen blocks start at
+  // any packed row; their copies start at the multiple of 4 below it (a tensor copy's
+  // first column must sit on 16 bytes) and are 132 columns wide to cover the block.
+  const uint32_t stat_box = varlen ? 132u : 128u;
+  CUtensorMap tl, td;
+  if ((rc = encode_vec_rows(&tl, lse2, seqlen_q, static_cast<uint64_t>(bm) * H,
+                            static_cast<uint64_t>(sq_pad) * 4, stat_box, "lse workspace")) != FA_OK)
     return rc;
-  if ((rc = encode_vec_rows(&td, dvec, seqlen_q, static_cast<uint64_t>(batch) * H,
-                            static_cast<uint64_t>(sq_pad) * 4, "D workspace")) != FA_OK)
+  if ((rc = encode_vec_rows(&td, dvec, seqlen_q, static_cast<uint64_t>(bm) * H,
+                            static_cast<uint64_t>(sq_pad) * 4, stat_box, "D workspace")) != FA_OK)
     return rc;
   fa::BwdParams p{};
   p.out = out;
@@ -725,11 +746,19 @@ int fa_bwd(const void* dout, const void* q, const void* k, const void* v, const 
   p.Hkv = Hkv;
   p.G = H / Hkv;
   p.scale = scale;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  float softcap_log2 = 0.f, tanh_k = 0.f, scale_log2 = 0.f;
+  fill_score_params(scale, softcap, &scale_log2, &softcap_log2, &tanh_k);
+  p.scale_log2 = scale_log2;
+  p.softcap_log2 = softcap_log2;
+  p.tanh_k = tanh_k;
   p.alibi = alibi_slopes;
   p.causal = causal ? 1 : 0;
   p.wl = window_left;
   p.wr = window_right;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.rows_q = rows_q;
+  p.rows_k = rows_k;
   p.status = status;
   p.timeout_ns = timeout_ns();
   const cudaError_t e = fa::launch_bwd(tq, tk, tv, tdo, tl, td, p, dtype == FA_BF16, d,

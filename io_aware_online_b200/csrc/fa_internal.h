@@ -62,10 +62,20 @@ struct DecodeParams {
   uint64_t timeout_ns;
   int sm_count;                    // persistent grid: CTAs per SM x sm_count (capped at items)
   unsigned int* item_counter;      // workspace word, zero at launch: next work item to claim
+  // longest-first order of the sequences (int16, in the workspace header after the
+  // counter), written by the prep kernel when B <= kDecOrderMax; NULL: natural order
+  const int16_t* order;
 };
+
+// Sequences the decode prep kernel ranks: the order fits the workspace's 256-byte
+// header after the counter (bytes 16 .. 255, int16 entries).
+constexpr int kDecOrderMax = 120;
 
 cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           bool bf16, int d, cudaStream_t stream);
+// Zeroes the decode's work-item counter and, when p.order is set, writes the
+// longest-first order of the sequences (one small CTA, before launch_decode).
+cudaError_t launch_decode_prep(const DecodeParams& p, cudaStream_t stream);
 
 // ---------------------------------------------------------------- KV append
 struct AppendParams {
@@ -100,7 +110,7 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 struct BwdParams {
   const void* out;                 // forward output O [B, Sq, H, D] (16-bit, contiguous)
   const void* dout;                // dO, same layout
-  const float* lse;                // [B, H, Sq] natural-log LSE of the forward
+  const float* lse;                // [B, H, Sq] (varlen [H, total_q]) natural-log LSE of the forward
   float* dvec;                     // [B, H, Sq] D = rowsum(dO * O) (workspace)
   float* lse2;                     // [B, H, Sq] LSE * log2(e) (workspace, after dvec)
   int sq_pad;                      // row stride of dvec / lse2: Sq rounded up to 4
@@ -110,8 +120,15 @@ struct BwdParams {
   int B, Sq, Sk, H, Hkv, G;
   float scale;                     // softmax_scale
   float scale_log2;                // softmax_scale * log2(e)
+  float softcap_log2;              // softcap * log2(e) (0: no softcap)
+  float tanh_k;                    // 2 * log2(e) * softmax_scale / softcap
   const float* alibi;              // [H] or NULL
   int causal, wl, wr;
+  // varlen (both non-NULL): sequence b owns rows cu_q[b] .. cu_q[b+1]-1 of the
+  // packed [total_q, H, D] tensors (Sq = total_q, B = number of sequences)
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int rows_q, rows_k;              // the grid's per-sequence extents (varlen: max_seqlen)
   unsigned int* status;
   uint64_t timeout_ns;
 };
@@ -119,6 +136,10 @@ struct BwdParams {
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tl, const CUtensorMap& td,
                        const BwdParams& p, bool bf16, int d, cudaStream_t stream);
+cudaError_t launch_bwd_varlen(const CUtensorMap& tq, const CUtensorMap& tk,
+                              const CUtensorMap& tv, const CUtensorMap& tdo,
+                              const CUtensorMap& tl, const CUtensorMap& td, const BwdParams& p,
+                              bool bf16, int d, cudaStream_t stream);
 
 cudaError_t launch_wait_timeout_selftest(unsigned int* status, uint64_t timeout_ns,
                                          cudaStream_t stream);

@@ -57,7 +57,8 @@ def attention_backward(q, k, v, do, *, scale=None, causal=False, window=(-1, -1)
                        softcap=0.0, alibi_slopes=None, return_probs=False):
     """q [B, Sq, H, d], k/v [B, Sk, Hkv, d], do like q.
     Returns (dq like q, dk, dv like k, o like q, lse [B, H, Sq]) in float64, and
-    with return_probs also P and dS [B, H, Sq, Sk]."""
+    with return_probs also P and dX [B, H, Sq, Sk] (the gradient with respect to
+    scale Q K^T: dS, times 1 - T^2 under a softcap)."""
     q, k, v, do = _np64(q), _np64(k), _np64(v), _np64(do)
     B, Sq, H, d = q.shape
     Sk, Hkv = k.shape[1], k.shape[2]
@@ -103,7 +104,7 @@ def attention_backward(q, k, v, do, *, scale=None, causal=False, window=(-1, -1)
             o[b, :, h] = O
             if return_probs:
                 probs[b, h] = P
-                dss[b, h] = dS
+                dss[b, h] = dX
             lse[b, h] = np.where(live, m[:, 0] + np.log(np.where(live, den[:, 0], 1.0)),
                                  -np.inf)
     if return_probs:

@@ -220,21 +220,24 @@ def test_fp8_validation(lib):
 
 def bwd(lib, **kw):
     a = dict(dout=P, q=P, k=P, v=P, out=P, lse=P, dq=P, dk=P, dv=P, dtype=1, B=1, Sq=256, Sk=256,
-             H=2, Hkv=2, d=128, scale=float("nan"), causal=1, wl=-1, wr=-1, softcap=0.0,
-             alibi=None, ws=P, ws_bytes=None, stream=None)
+             H=2, Hkv=2, d=128, cuq=None, cuk=None, mq=0, mk=0, scale=float("nan"), causal=1,
+             wl=-1, wr=-1, softcap=0.0, alibi=None, ws=P, ws_bytes=None, stream=None)
     a.update(kw)
     if a["ws_bytes"] is None:
-        a["ws_bytes"] = lib.fa_bwd_workspace_size(a["B"], a["Sq"], a["H"])
+        a["ws_bytes"] = lib.fa_bwd_workspace_size(1 if a["cuq"] else a["B"], a["Sq"], a["H"])
     return lib.fa_bwd(a["dout"], a["q"], a["k"], a["v"], a["out"], a["lse"], a["dq"], a["dk"],
                       a["dv"], a["dtype"], a["B"], a["Sq"], a["Sk"], a["H"], a["Hkv"], a["d"],
-                      a["scale"], a["causal"], a["wl"], a["wr"], a["softcap"], a["alibi"],
-                      a["ws"], a["ws_bytes"], a["stream"])
+                      a["cuq"], a["cuk"], a["mq"], a["mk"], a["scale"], a["causal"], a["wl"],
+                      a["wr"], a["softcap"], a["alibi"], a["ws"], a["ws_bytes"], a["stream"])
 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(d=96), FA_ERR_UNSUPPORTED),
     (dict(dtype=2), FA_ERR_UNSUPPORTED),
-    (dict(softcap=30.0), FA_ERR_UNSUPPORTED),               # no softcap in the backward
+    (dict(softcap=-1.0), FA_ERR_INVALID_ARG),
+    (dict(cuq=P), FA_ERR_INVALID_ARG),                      # varlen needs both offsets
+    (dict(cuq=P, cuk=P, mq=300), FA_ERR_INVALID_ARG),      # max_seqlen above the total
+    (dict(cuq=P, cuk=P, mq=200, mk=-1), FA_ERR_INVALID_ARG),
     (dict(H=3, Hkv=2), FA_ERR_INVALID_ARG),
     (dict(dout=None), FA_ERR_INVALID_ARG),
     (dict(lse=None), FA_ERR_INVALID_ARG),
@@ -263,6 +266,13 @@ def test_bwd_workspace_size(lib):
 
 def test_bwd_empty_batch_is_a_noop(lib):
     assert bwd(lib, B=0) == FA_OK
+
+
+def test_bwd_varlen_workspace_is_one_packed_entry(lib):
+    # varlen: the statistics cover [num_heads, total_q]; a workspace sized for the
+    # packed rows passes the check (an empty batch then returns before any launch)
+    assert bwd(lib, B=0, cuq=P, cuk=P, mq=100, mk=100) == FA_OK
+    assert bwd(lib, B=3, cuq=P, cuk=P, mq=100, mk=100, ws_bytes=16) == FA_ERR_WORKSPACE
 
 
 def test_binding_refuses_host_tensors(lib):

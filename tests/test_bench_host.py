@@ -35,7 +35,7 @@ def test_decode_bytes_counts_valid_tokens_only():
     kv = sum(lens) * c["Hkv"] * c["d"] * 2 * 2
     io = c["B"] * c["Sq"] * c["H"] * c["d"] * 2 * 2 + c["B"] * c["H"] * c["Sq"] * 4
     bt = (1 + 1 + 2) * 4 + c["B"] * 4      # pages touched, plus cache_seqlens
-    assert bench.decode_bytes(lens, 16) == kv + io + bt
+    assert bench.decode_bytes(lens) == kv + io + bt
 
 
 def test_clock_summary_parses_reasons_and_ignores_idle_samples():
@@ -75,3 +75,17 @@ def test_profiled_traffic_follows_the_source_hash(tmp_path, monkeypatch):
     assert bench.profiled_traffic("k.md", ["a.cuh", "b.cu"]) is None
     assert bench.profiled_traffic("missing.md", ["a.cuh"]) is None
 
+
+
+def test_stats_report_median_min_and_mean():
+    st = bench._stats([3.0, 1.0, 2.0, 10.0])
+    assert st["median_ms"] == 2.5 and st["min_ms"] == 1.0 and st["mean_ms"] == 4.0
+    assert st["launch_samples"] == 4
+
+
+def test_max_abs_requires_the_same_infinities():
+    import math
+    assert bench._max_abs([1.0, 2.0], [1.5, 2.0]) == 0.5
+    assert bench._max_abs([-math.inf, 1.0], [-math.inf, 1.25]) == 0.25
+    # a -inf LSE on one side only is a mismatch, reported as an infinite difference
+    assert bench._max_abs([0.0, 1.0], [-math.inf, 1.0]) == math.inf

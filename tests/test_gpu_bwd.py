@@ -8,10 +8,12 @@ fp32 accumulation and the approximate exp2):
 
     dD_i  = u * sum_c |dO_ic| |O_ic|                  (D from the rounded O)
     |ddV| <= u * sum_i P_ij |dO_ic|  + u |dV|          (P rounded before P^T dO)
-    |ddK| <= scale * sum_i (u |dS_ij| + P_ij dD_i) |Q_ic| + u |dK|
-    |ddQ| <= scale * sum_j (u |dS_ij| + P_ij dD_i) |K_jc| + u |dQ|
+    |ddK| <= scale * sum_i (u |dX_ij| + P_ij dD_i) |Q_ic| + u |dK|
+    |ddQ| <= scale * sum_j (u |dX_ij| + P_ij dD_i) |K_jc| + u |dQ|
 
-P and dS are the oracle's exact values.
+P and dX (the gradient with respect to scale Q K^T: dS, times 1 - tanh^2 under a
+softcap, whose factor is at most 1) are the oracle's exact values.  Varlen cases
+take these bounds sequence by sequence.
 """
 import numpy as np
 import pytest
@@ -147,3 +149,100 @@ def test_forward_then_backward_matches_oracle():
     for name, got, ref in (("dq", dq, dq_r), ("dk", dk, dk_r), ("dv", dv, dv_r)):
         rel = np.linalg.norm(f64(got) - ref) / np.linalg.norm(ref)
         assert rel <= 1e-2, f"{name}: relative error {rel:.3g}"
+
+
+def test_softcap_causal_bf16_d128():
+    """softcap 2: most scores sit on the curved part of c tanh(x / c)."""
+    run_case(1, 384, 384, 4, 2, 128, torch.bfloat16, 1810, causal=True, softcap=2.0)
+
+
+def test_softcap_alibi_window_fp16_d64():
+    run_case(1, 320, 320, 4, 4, 64, torch.float16, 1811, causal=True, window_size=(150, -1),
+             softcap=3.0, alibi_slopes=synth.alibi_slopes(4))
+
+
+def run_varlen(lq, lk, H, Hkv, d, dtype, seed, **kw):
+    """Packed sequences (section 3.2): each sequence against the dense oracle on its
+    own rows, with that sequence's bounds."""
+    g = torch.Generator().manual_seed(seed)
+    tq, tk = sum(lq), sum(lk)
+    q = synth.randn((tq, H, d), dtype, g)
+    k = synth.randn((tk, Hkv, d), dtype, g)
+    v = synth.randn((tk, Hkv, d), dtype, g)
+    do = synth.randn((tq, H, d), dtype, g)
+    cu_q, cu_k = synth.cu_seqlens(lq), synth.cu_seqlens(lk)
+    okw = {("window" if kk == "window_size" else kk): vv for kk, vv in kw.items()}
+    o_r, l_r = np.zeros((tq, H, d)), np.full((H, tq), -np.inf)
+    refs = []
+    for b in range(len(lq)):
+        qa, qb, ka, kb = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if qb == qa or kb == ka:
+            refs.append(None)
+            continue
+        r = oracle.attention_backward(q[None, qa:qb], k[None, ka:kb], v[None, ka:kb],
+                                      do[None, qa:qb], return_probs=True, **okw)
+        refs.append(r)
+        o_r[qa:qb], l_r[:, qa:qb] = r[3][0], r[4][0]
+    o16 = torch.from_numpy(o_r).to(dtype)
+    dkw = dict(kw)
+    if dkw.get("alibi_slopes") is not None:
+        dkw["alibi_slopes"] = dkw["alibi_slopes"].to(DEV)
+    dq, dk, dv = fa().fa_bwd(do.to(DEV), q.to(DEV), k.to(DEV), v.to(DEV), o16.to(DEV),
+                             torch.from_numpy(l_r).float().contiguous().to(DEV),
+                             cu_seqlens_q=cu_q.to(DEV), cu_seqlens_k=cu_k.to(DEV),
+                             max_seqlen_q=max(lq), max_seqlen_k=max(lk), **dkw)
+    torch.cuda.synchronize()
+    sc = d ** -0.5
+    for b, r in enumerate(refs):
+        qa, qb, ka, kb = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if r is None:
+            # no keys or no queries: the gradients of the sequence's rows are zero
+            assert torch.all(dq[qa:qb].float() == 0) and torch.all(dk[ka:kb].float() == 0)
+            assert torch.all(dv[ka:kb].float() == 0)
+            continue
+        dq_r, dk_r, dv_r, _, _, P, dX = r
+        tq_, tk_, tv_ = bounds(q[None, qa:qb], k[None, ka:kb], do[None, qa:qb],
+                               f64(o16[None, qa:qb]), P, dX, dq_r, dk_r, dv_r, sc, H // Hkv,
+                               U[dtype])
+        check(f"dq[seq {b}]", dq[None, qa:qb], dq_r, tq_)
+        check(f"dk[seq {b}]", dk[None, ka:kb], dk_r, tk_)
+        check(f"dv[seq {b}]", dv[None, ka:kb], dv_r, tv_)
+
+
+def test_varlen_causal_bf16_d128():
+    # lengths off the 128 grid, more keys than queries, a one-row sequence, and a
+    # sequence longer than two blocks
+    run_varlen([1, 130, 300, 64], [1, 257, 300, 200], 4, 2, 128, torch.bfloat16, 1820,
+               causal=True)
+
+
+def test_varlen_softcap_window_fp16_d64():
+    run_varlen([200, 77, 129], [200, 150, 129], 4, 4, 64, torch.float16, 1821, causal=True,
+               window_size=(64, -1), softcap=5.0)
+
+
+def test_varlen_matches_dense_per_sequence_bitwise():
+    """A packed batch gives, row for row, the bits of separate dense calls."""
+    lq = [150, 260]
+    g = torch.Generator().manual_seed(1822)
+    H, d, dt = 2, 64, torch.bfloat16
+    q, k, v, do = (synth.randn((sum(lq), H, d), dt, g) for _ in range(4))
+    cu = synth.cu_seqlens(lq)
+    qd, kd, vd, dod = q.to(DEV), k.to(DEV), v.to(DEV), do.to(DEV)
+    out, lse = fa().fa_fwd(qd, kd, vd, cu_seqlens_q=cu.to(DEV), cu_seqlens_k=cu.to(DEV),
+                           max_seqlen_q=max(lq), max_seqlen_k=max(lq), causal=True)
+    dq, dk, dv = fa().fa_bwd(dod, qd, kd, vd, out, lse, cu_seqlens_q=cu.to(DEV),
+                             cu_seqlens_k=cu.to(DEV), max_seqlen_q=max(lq),
+                             max_seqlen_k=max(lq), causal=True)
+    for b in range(len(lq)):
+        a, e = int(cu[b]), int(cu[b + 1])
+        sl = slice(a, e)
+        # the same forward outputs, sliced: only the backward is compared
+        o1 = out[None, sl].contiguous()
+        l1 = lse[:, sl][None].contiguous()
+        g1 = fa().fa_bwd(dod[None, sl].contiguous(), qd[None, sl].contiguous(),
+                         kd[None, sl].contiguous(), vd[None, sl].contiguous(), o1, l1,
+                         causal=True)
+        torch.cuda.synchronize()
+        for name, x, y in (("dq", dq, g1[0]), ("dk", dk, g1[1]), ("dv", dv, g1[2])):
+            assert torch.equal(x[sl], y[0]), f"{name}: sequence {b} differs from its dense call"
