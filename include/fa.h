@@ -109,6 +109,41 @@ FA_API int fa_fwd(const void *q, const void *k, const void *v, void *out, float 
            int window_right, float softcap, const float *alibi_slopes, void *stream);
 
 /*
+ * fa_fwd_host -- fa_fwd (dense, section 3.1 flash_attn_func) on operands in host
+ * memory, with the transfers overlapped with the kernels.
+ *
+ *   q [batch, seqlen_q, num_heads, head_dim], k/v [batch, seqlen_k, num_heads_k,
+ *   head_dim], out like q: contiguous, fp16 or bf16 (dtype), in host memory;
+ *   lse fp32 [batch, num_heads, seqlen_q] in host memory, or NULL; alibi_slopes
+ *   fp32 [num_heads] in host memory, or NULL.  Page-locked memory (cudaHostAlloc,
+ *   cudaHostRegister) lets the copies run asynchronously and overlap; pageable
+ *   memory works but each copy then waits on the host.
+ *   workspace: device memory, 256-byte aligned, at least
+ *   fa_fwd_host_workspace_size(batch, seqlen_q, seqlen_k, num_heads, num_heads_k,
+ *   head_dim, lse != NULL) bytes; owned by the caller, who keeps it (and the host
+ *   buffers) alive until `stream` has passed the call.
+ * The batch is cut into at most four chunks of whole sequences that pass through
+ * two workspace slots: chunk c+1 is copied in and chunk c-1 copied out while chunk c
+ * is computed, on three streams of the library that start after the work already
+ * on `stream` and that `stream` waits for at the end of the call.  Results are
+ * bit-identical to fa_fwd over the whole batch.  Masks, scale and softcap as for
+ * fa_fwd (varlen, strides and FP8 are not offered here).
+ * Errors: argument and workspace errors return FA_ERR_* before anything is enqueued;
+ * an error from a later step returns after `stream` has been made to wait for what
+ * was enqueued, and out / lse are then undefined.  Calls from several host threads
+ * are serialised while they enqueue; the streams are created on a device's first
+ * call and kept for the life of the process (not valid after a device reset).
+ */
+FA_API size_t fa_fwd_host_workspace_size(int batch, int seqlen_q, int seqlen_k, int num_heads,
+                                         int num_heads_k, int head_dim, int with_lse);
+FA_API int fa_fwd_host(const void *q, const void *k, const void *v, void *out, float *lse,
+                       int dtype, int batch, int seqlen_q, int seqlen_k, int num_heads,
+                       int num_heads_k, int head_dim, float softmax_scale, int causal,
+                       int window_left, int window_right, float softcap,
+                       const float *alibi_slopes, void *workspace, size_t workspace_bytes,
+                       void *stream);
+
+/*
  * fa_fwd_fp8 -- fa_fwd with 8-bit inputs (the "FlashAttention common interfaces"
  * page's workflow three: q, k and v cast to float8 E4M3 and passed to the same
  * call; FlashAttention-3's FP8 path on the tag page).

@@ -8,6 +8,8 @@ library is missing or a call fails, an exception is raised.
 
 Functions mirror include/fa.h:
     fa_fwd(q, k, v, ...)                  dense [B,S,H,d] or varlen [total,H,d]
+    fa_fwd_host(q, k, v, ...)             dense, q/k/v/out in host memory (transfers
+                                          overlapped with the kernels)
     fa_fwd_kvcache(q, k_cache, v_cache, ...)
     fa_fwd_kvcache_static(q, k_cache, v_cache, ...)   (no workspace; fixed device scratch)
     fa_combine(out_partial, lse_partial, ...)
@@ -22,7 +24,7 @@ import os
 
 import torch
 
-__all__ = ["FAError", "fa_fwd", "fa_fwd_kvcache", "fa_fwd_kvcache_static", "fa_combine",
+__all__ = ["FAError", "fa_fwd", "fa_fwd_host", "fa_fwd_host_workspace_size", "fa_fwd_kvcache", "fa_fwd_kvcache_static", "fa_combine",
            "fa_kvcache_num_splits",
            "fa_kvcache_workspace_size", "fa_device_status", "fa_set_wait_timeout_ms",
            "fa_version", "library_path", "load"]
@@ -62,6 +64,11 @@ def load():
                                i64p, i64p, i64p, i64p, vp, vp, i32, i32, f32, i32, i32, i32, f32,
                                vp, vp]
     lib.fa_fwd_fp8.restype = i32
+    lib.fa_fwd_host_workspace_size.argtypes = [i32] * 7
+    lib.fa_fwd_host_workspace_size.restype = ctypes.c_size_t
+    lib.fa_fwd_host.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+                                i32, i32, f32, vp, vp, ctypes.c_size_t, vp]
+    lib.fa_fwd_host.restype = i32
     lib.fa_kvcache_num_splits.argtypes = [i32] * 8
     lib.fa_kvcache_num_splits.restype = i32
     lib.fa_kvcache_workspace_size.argtypes = [i32] * 8
@@ -208,6 +215,51 @@ def fa_fwd(q, k, v, *, out=None, lse=None, cu_seqlens_q=None, cu_seqlens_k=None,
     else:
         _check(lib.fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), *fp8, B, sq, sk,
                               H, Hkv, d, *args))
+    return out, lse
+
+
+def _host_ptr(t) -> ctypes.c_void_p | None:
+    """Address of a contiguous CPU tensor (page-locked ones let the copies overlap)."""
+    if t is None:
+        return None
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("fa_fwd_host takes contiguous CPU tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def fa_fwd_host_workspace_size(batch, seqlen_q, seqlen_k, num_heads, num_heads_k, head_dim,
+                               with_lse=True) -> int:
+    return int(load().fa_fwd_host_workspace_size(batch, seqlen_q, seqlen_k, num_heads,
+                                                 num_heads_k, head_dim, int(bool(with_lse))))
+
+
+def fa_fwd_host(q, k, v, *, out=None, lse=None, softmax_scale=None, causal=False,
+                window_size=(-1, -1), softcap=0.0, alibi_slopes=None, return_lse=True,
+                workspace=None, stream=None):
+    """fa_fwd on dense q [B, Sq, H, d], k/v [B, Sk, Hkv, d] in host memory; out (and lse
+    [B, H, Sq], and alibi_slopes [H]) in host memory too.  The library copies the batch
+    through a device workspace (on the current CUDA device) chunk by chunk, overlapping
+    the copies with the kernels.  When `stream` (default: the current stream) has passed
+    the call, out and lse hold the results."""
+    lib = load()
+    dt = _dtype(q)
+    B, sq, H, d = q.shape
+    sk, Hkv = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, sq), dtype=torch.float32, pin_memory=True)
+    if workspace is None:
+        n = fa_fwd_host_workspace_size(B, sq, sk, H, Hkv, d, lse is not None)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8,
+                                device=torch.device("cuda", torch.cuda.current_device()))
+    if alibi_slopes is not None and (alibi_slopes.is_cuda or alibi_slopes.dtype != torch.float32):
+        raise ValueError("fa_fwd_host takes fp32 CPU alibi_slopes")
+    _check(lib.fa_fwd_host(_host_ptr(q), _host_ptr(k), _host_ptr(v), _host_ptr(out),
+                           _host_ptr(lse), dt, B, sq, sk, H, Hkv, d, _scale(softmax_scale),
+                           int(bool(causal)), int(window_size[0]), int(window_size[1]),
+                           float(softcap), _host_ptr(alibi_slopes), _ptr(workspace),
+                           workspace.numel(), _stream(stream)))
     return out, lse
 
 

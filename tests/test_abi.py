@@ -152,6 +152,38 @@ def test_static_scratch_validation(lib):
     assert lib.fa_kvcache_static_scratch_bytes() == 24 << 20
 
 
+def test_host_entry_validation(lib):
+    # argument and workspace errors come back before any device use
+    h = lib.fa_fwd_host
+    ws = lib.fa_fwd_host_workspace_size(4, 256, 256, 8, 2, 64, 1)
+    # 256 B of slopes, then two slots of one sequence each: q, k, v, out, lse
+    q1, kv1, l1 = 256 * 8 * 64 * 2, 256 * 2 * 64 * 2, 8 * 256 * 4
+    assert ws == 256 + 2 * (2 * q1 + 2 * kv1 + l1)
+    assert lib.fa_fwd_host_workspace_size(4, 256, 256, 8, 2, 64, 0) == 256 + 2 * (2 * q1 + 2 * kv1)
+    assert lib.fa_fwd_host_workspace_size(0, 256, 256, 8, 2, 64, 1) == 0
+    # B=9: chunks of 3 sequences
+    assert lib.fa_fwd_host_workspace_size(9, 128, 128, 1, 1, 128, 0) == \
+        256 + 2 * (2 * 3 * 128 * 128 * 2 + 2 * 3 * 128 * 128 * 2)
+    W = ctypes.c_void_p(1 << 20)  # never dereferenced: every case fails validation first
+    good = [P, P, P, P, None, 0, 4, 256, 256, 8, 2, 64, float("nan"), 1, -1, -1, 0.0, None]
+    ws0 = lib.fa_fwd_host_workspace_size(4, 256, 256, 8, 2, 64, 0)  # lse is NULL below
+    def call(args, ws_ptr=W, ws_bytes=ws0):
+        return h(*args, ws_ptr, ws_bytes, None)
+    bad = list(good); bad[0] = None
+    assert call(bad) == FA_ERR_INVALID_ARG
+    bad = list(good); bad[5] = 2                                   # fp32 inputs
+    assert call(bad) == FA_ERR_UNSUPPORTED
+    bad = list(good); bad[10] = 3                                  # 8 heads over 3 KV heads
+    assert call(bad) == FA_ERR_INVALID_ARG
+    bad = list(good); bad[11] = 96
+    assert call(bad) == FA_ERR_UNSUPPORTED
+    assert call(good, ws_bytes=ws0 - 1) == FA_ERR_WORKSPACE
+    assert call(good, ws_ptr=None) == FA_ERR_WORKSPACE
+    assert call(good, ws_ptr=ctypes.c_void_p((1 << 20) + 16)) == FA_ERR_WORKSPACE  # alignment
+    empty = list(good); empty[6] = 0
+    assert call(empty) == FA_OK                                    # nothing to do
+
+
 def test_combine_validation(lib):
     assert lib.fa_combine(P, P, P, None, 0, 1, 1, 1, 64, 0, None, None, None) == FA_ERR_INVALID_ARG
     assert lib.fa_combine(P, P, P, None, 0, 1, 1, 1, 64, 300, None, None, None) == FA_ERR_INVALID_ARG
