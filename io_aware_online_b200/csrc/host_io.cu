@@ -30,7 +30,7 @@
 
 namespace {
 
-constexpr int kMaxDev = 64;
+constexpr int kPipeMaxDev = 64;
 constexpr int kMaxChunks = 4;  // the batch is cut into at most this many chunks
 constexpr size_t kAlign = 256;
 
@@ -41,7 +41,7 @@ struct HostPipe {
 };
 
 std::mutex g_host_mu;
-HostPipe g_pipe[kMaxDev];
+HostPipe g_pipe[kPipeMaxDev];
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -67,7 +67,7 @@ int chunk_batch(int batch) {
 
 int pipe_of_current_device(HostPipe** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kPipeMaxDev)
     return fa::set_error(FA_ERR_CUDA, "fa_fwd_host: no usable current CUDA device");
   HostPipe& p = g_pipe[dev];
   if (!p.ready) {
