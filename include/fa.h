@@ -159,7 +159,7 @@ FA_API int fa_fwd_host(const void *q, const void *k, const void *v, void *out, f
  * relative error of at most 2^-4, and O differs from exact attention on the
  * dequantised inputs by at most 2^-4 * sum_j w_ij |v_j| per element (w the exact
  * attention weights) plus n_k * 2^-18 * max_j |v_j| (probabilities below 2^-14 of
- * the row's largest fall in E4M3's subnormal range), plus the bf16 rounding of O.
+ * the row's largest can fall in E4M3's subnormal range), plus the bf16 rounding of O.
  * The LSE comes from the exact fp32 sum.  Other arguments, masks and errors as for
  * fa_fwd.
  */

@@ -9,13 +9,19 @@ cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const C
   if (d != 128) return cudaErrorInvalidValue;
   const bool sc = p.softcap_log2 > 0.f;
   const bool al = p.alibi != nullptr;
-#define FA_FWD8_CASE(SC, AL)                                                               \
-  if (sc == SC && al == AL)                                                                \
-    return launch_fwd_inst<128, 2, true, SC, AL, 0, true>(tq, tk, tv, p, batch, rows_q, stream);
-  FA_FWD8_CASE(false, false)
-  FA_FWD8_CASE(true, false)
-  FA_FWD8_CASE(false, true)
-  FA_FWD8_CASE(true, true)
+  // exponential pairs (of 8) on the FMA pipe: the 8-bit path is bound by the
+  // exponentials (its products take half the bf16 time); FA_EXP2_EMU overrides
+  const int emu = (sc || al) ? 0 : fp8_exp2_emu_choice();
+#define FA_FWD8_CASE(SC, AL, EM)                                                           \
+  if (sc == SC && al == AL && emu == EM)                                                   \
+    return launch_fwd_inst<128, 2, true, SC, AL, EM, true>(tq, tk, tv, p, batch, rows_q, stream);
+  FA_FWD8_CASE(false, false, 0)
+  FA_FWD8_CASE(false, false, 2)
+  FA_FWD8_CASE(false, false, 3)
+  FA_FWD8_CASE(false, false, 4)
+  FA_FWD8_CASE(true, false, 0)
+  FA_FWD8_CASE(false, true, 0)
+  FA_FWD8_CASE(true, true, 0)
 #undef FA_FWD8_CASE
   return cudaErrorInvalidValue;
 }

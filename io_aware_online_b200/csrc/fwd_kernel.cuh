@@ -60,10 +60,15 @@ constexpr uint32_t kSoftmaxRegs = 200;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
-// 8-bit P: the running max is kept exact (any growth rescales O) and P is taken
-// against max - 8, so P lies in (0, 256] (E4M3 tops out at 448) and values down to
-// 2^-17 of the row's largest stay in E4M3's normal range instead of underflowing.
+// 8-bit P is taken against the running max minus 8, and the running max is lazy
+// with a threshold of 0.8 (log2 units): P then stays at or below 2^8.8 < 448, the
+// largest E4M3 value, and a probability is subnormal in E4M3 only below 2^-14 of
+// the row's largest (2^-14.8 when the running max is 0.8 stale), so the error bound
+// of an exact running max holds.  (With an exact max, O was rescaled in most
+// blocks: for random scores some row of a warp raises its max at almost every
+// block.)
 constexpr float kP8Offset = 8.0f;
+constexpr float kP8Threshold = 0.8f;
 
 // T query tiles per CTA (1 or 2).  With T = 2 one CTA fills an SM (512 TMEM
 // columns, 12 warps); with T = 1 two CTAs share an SM (256 columns and 8 warps
@@ -705,7 +710,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T, FP8 ? 1 : 2>::kThreads,
       // stay in registers until that check.  Warps with a row that has not met an
       // allowed key yet (running max -inf) take the max-first order.
       const bool spec = !Cfg::kSepP && !FP8 && __all_sync(0xffffffffu, m_use != -INFINITY);
-      constexpr float kThreshold = FP8 ? 0.f : kRescaleThreshold;
+      constexpr float kThreshold = FP8 ? kP8Threshold : kRescaleThreshold;
       bool need = false;
       float alpha = 1.f;
       auto update_max = [&](float m_blk) {

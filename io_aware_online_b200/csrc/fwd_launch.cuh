@@ -61,6 +61,16 @@ inline int fwd_tiles_choice() {
   return 2;
 }
 
+// The same choice for the 8-bit path (default 2).
+inline int fp8_exp2_emu_choice() {
+  static const int env = [] {
+    const char* e = std::getenv("FA_EXP2_EMU");
+    return e ? std::atoi(e) : -1;
+  }();
+  if (env == 0 || env == 2 || env == 3 || env == 4) return env;
+  return 2;
+}
+
 template <bool BF16>
 cudaError_t launch_fwd_dtype(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const FwdParams& p, int d, int batch, int rows_q,
