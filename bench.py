@@ -585,7 +585,12 @@ def run_fp8(args, rank, world, local):
                        "untimed)", "parallelism": f"dp{world} (independent replicas)"},
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": fp8_peak,
                          "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
-                         "traffic": None,
+                         "traffic": (profiled_traffic("fwd_kernel_fp8_causal_B4_S8192.md",
+                                                      ["fwd_kernel.cuh", "fwd_launch.cuh",
+                                                       "fwd_fp8.cu", "sm100.cuh",
+                                                       "fa_internal.h"])
+                                     # the capture ran the default exponential split
+                                     if os.environ.get("FA_EXP2_EMU") is None else None),
                          "kernel": "fwd_kernel<128, 2 tiles, e4m3, causal> (kind::f8f6f4)",
                          "peak_source": f"{peak_src} bf16 burst x 2 (nominal e4m3/bf16 ratio)"},
             "gpu_launches": K, "clocks": clk.summary()}
