@@ -68,9 +68,8 @@ struct BwdCfg {
   static constexpr int kStat = kStage + 4 * kTileBytes;
   static constexpr int kBarOff = kStat + 2 * 2 * kStatPitch * 4;
   static_assert(kStat % 128 == 0 && (kStatPitch * 4) % 128 == 0, "tensor copy destinations");
-  // fix_full, full[2], empty[2], s_full, p_full, s_read, dp_read, done, drain, dp_full,
-  // ds_full
-  static constexpr int kNumBars = 13;
+  // fix_full, full[2], empty[2], s_full, p_full, done, drain, dp_full, ds_full
+  static constexpr int kNumBars = 11;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   // room to align the base to 1 KiB; at least 116 KiB, so that one CTA fills an SM
@@ -96,8 +95,8 @@ struct DqCfg {
   static constexpr int kV = kK + kKStages * kTileBytes;
   static constexpr int kBarOff = kV + kVStages * kTileBytes;
   // fix_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, p_full[2],
-  // s_read[2], dp_read, done, drain, dp_full
-  static constexpr int kNumBars = 20;
+  // dp_read, done, drain, dp_full
+  static constexpr int kNumBars = 18;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc =
@@ -223,6 +222,19 @@ static_assert(256 * kBwdComputeRegs + 128 * kBwdOtherRegs == kWideThreads * kBwd
 
 // One CTA per (128-key block kb, KV head hk, batch b).
 
+// O (+)= A B, A (16-bit, 128 keys or queries along K) from tensor memory in two runs
+// of 32 columns: [a, a + 32) holds K-steps 0..63 and [a + 64, a + 96) K-steps
+// 64..127, because each compute warpgroup writes its 16-bit values over its own
+// 64 score columns.  B MN-major as in fwd_issue_pv (16 rows = 2 KiB a step).
+__device__ __forceinline__ void bwd_issue_split_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
+                                                  uint32_t idesc, bool acc) {
+  const uint32_t b_lo = static_cast<uint32_t>(b0), b_hi = static_cast<uint32_t>(b0 >> 32);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ts(d_tmem, a_tmem + (kk / 4) * 64 + (kk % 4) * 8, desc_pack(b_lo + kk * (2048 >> 4), b_hi),
+           idesc, (acc || kk > 0) ? 1u : 0u);
+}
+
 template <int D, bool BF16, bool ALIBI, bool SOFTCAP, bool VARLEN>
 __global__ void __launch_bounds__(kWideThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -261,12 +273,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   uint64_t* empty = bars + 3;
   uint64_t* s_full = bars + 5;
   uint64_t* p_full = bars + 6;
-  uint64_t* s_read = bars + 7;   // warpgroup 0 holds its S^T columns in registers
-  uint64_t* dp_read = bars + 8;  // ... and its dP^T columns
-  uint64_t* done = bars + 9;
-  uint64_t* drain = bars + 10;
-  uint64_t* dp_full = bars + 11;
-  uint64_t* ds_full = bars + 12;
+  uint64_t* done = bars + 7;
+  uint64_t* drain = bars + 8;
+  uint64_t* dp_full = bars + 9;
+  uint64_t* ds_full = bars + 10;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -280,8 +290,6 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     mbar_init(dp_full, 1);
     mbar_init(p_full, 8);   // one arrival per compute warp
     mbar_init(ds_full, 8);
-    mbar_init(s_read, 4);   // the four warps of warpgroup 0
-    mbar_init(dp_read, 4);
     mbar_init(done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -374,8 +382,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         if (!(ok = wait_bounded(p_full, n & 1, w))) break;
         tc_fence_after();
         // B operands MN-major: rows are queries, the head dim contiguous
-        fwd_issue_pv<D>(tbase + 256, tbase, sw128_desc(sdo, Cfg::kChunkBytes, 1024), idesc_acc,
-                        n > 0);                                                   // dV(n)
+        bwd_issue_split_a(tbase + 256, tbase, sw128_desc(sdo, Cfg::kChunkBytes, 1024), idesc_acc,
+                          n > 0);                                                 // dV(n)
         if (more) {
           if (!(ok = wait_bounded(full + (s ^ 1), ((n + 1) >> 1) & 1, w))) break;
           tc_fence_after();
@@ -384,8 +392,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         }
         if (!(ok = wait_bounded(ds_full, n & 1, w))) break;
         tc_fence_after();
-        fwd_issue_pv<D>(tbase + 256 + D, tbase + 128, sw128_desc(sq, Cfg::kChunkBytes, 1024),
-                        idesc_acc, n > 0);                                        // dK(n)
+        bwd_issue_split_a(tbase + 256 + D, tbase + 128, sw128_desc(sq, Cfg::kChunkBytes, 1024),
+                          idesc_acc, n > 0);                                      // dK(n)
         tc_commit(empty + s);
         if (more) {
           fwd_issue_qk<D>(tbase + 128, dVk,
@@ -431,8 +439,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           return *reinterpret_cast<const float4*>(a);
       };
       // phase 1: P^T of this half (fp32 in registers), 16-bit copy to columns
-      // [32 cg, 32 cg + 32), which hold S^T columns of warpgroup 0: warpgroup 1
-      // stores only once warpgroup 0 has its scores in registers
+      // [64 cg, 64 cg + 32), over this warpgroup's own S^T columns
       const bool open = mg.tile_open(qb, k0);  // uniform: the whole tile is unmasked
       float pf[64];
       uint32_t gh[SOFTCAP ? 32 : 1];  // softcap: 1 - tanh^2 per element, f16 pairs
@@ -442,11 +449,6 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         tmem_ld32(tbase + cg * 64 + 32 + lane_off, sv + 32);
         tmem_ld_wait(sv);
         tmem_ld_wait(sv + 32);
-        if (cg == 0) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(s_read);
-        }
 
         // every exponential is taken and a masked one then dropped by a select: a
         // branch per element would split the loop into blocks of one exponential
@@ -493,26 +495,18 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         else
           probs(std::true_type{});
       }
-      if (cg == 1) {
-        ok = wait_bounded(s_read, n & 1, w);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-      }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pp[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) pp[e] = pack2<BF16>(pf[c * 32 + 2 * e], pf[c * 32 + 2 * e + 1]);
-        tmem_st16(tbase + cg * 32 + c * 16 + lane_off, pp);
+        tmem_st16(tbase + cg * 64 + c * 16 + lane_off, pp);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      // phase 2: dS^T = P^T * (dP^T - D), the same column split over dP^T
+      // phase 2: dS^T = P^T * (dP^T - D), 16-bit over this warpgroup's own dP^T columns
       ok = wait_bounded(dp_full, n & 1, w);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
@@ -525,11 +519,6 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         tmem_ld32(tbase + 128 + cg * 64 + 32 + lane_off, dp + 32);
         tmem_ld_wait(dp);
         tmem_ld_wait(dp + 32);
-        if (cg == 0) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(dp_read);
-        }
 #pragma unroll
         for (int e = 0; e < 64; e += 4) {
           const float4 d4 = ld4(dd + e);
@@ -546,20 +535,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           }
         }
       }
-      if (cg == 1) {
-        ok = wait_bounded(dp_read, n & 1, w);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-      }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t ps[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) ps[e] = pack2<BF16>(pf[c * 32 + 2 * e], pf[c * 32 + 2 * e + 1]);
-        tmem_st16(tbase + 128 + cg * 32 + c * 16 + lane_off, ps);
+        tmem_st16(tbase + 128 + cg * 64 + c * 16 + lane_off, ps);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -657,12 +638,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   // alternating pairs, by block parity: an arrival for block j+2 needs the other
   // side to have finished block j, so neither runs two phases ahead of its waiter
   uint64_t* p_full[2] = {s_full + 1, s_full + 2};   // dS of the block written
-  uint64_t* s_read[2] = {s_full + 3, s_full + 4};   // warpgroup 0 holds its S columns
-  uint64_t* dp_read = s_full + 5;  // every compute warp holds its dP columns in registers
-  uint64_t* done = s_full + 6;
-  uint64_t* drain = s_full + 7;
-  uint64_t* dp_full = s_full + 8;
-  static_assert(1 + 2 * KS + 2 * VS + 9 == Cfg::kNumBars, "barrier count");
+  uint64_t* dp_read = s_full + 3;  // every compute warp holds its dP columns in registers
+  uint64_t* done = s_full + 4;
+  uint64_t* drain = s_full + 5;
+  uint64_t* dp_full = s_full + 6;
+  static_assert(1 + 2 * KS + 2 * VS + 7 == Cfg::kNumBars, "barrier count");
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -677,10 +657,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       mbar_init(v_empty + s, 1);
     }
     mbar_init(s_full, 1);
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(p_full[x], 8);  // dS written: one arrival per compute warp
-      mbar_init(s_read[x], 4);  // the four warps of warpgroup 0
-    }
+    for (int x = 0; x < 2; ++x) mbar_init(p_full[x], 8);  // dS written: one arrival per compute warp
     mbar_init(dp_full, 1);
     mbar_init(dp_read, 8);
     mbar_init(done, 1);
@@ -785,8 +762,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         if (!(ok = wait_bounded(p_full[s], (it >> 1) & 1, w))) break;
         tc_fence_after();
         // dQ += dS K_j: B = K_j MN-major (rows are keys, the head dim contiguous)
-        fwd_issue_pv<D>(tbase + 384, tbase + s * 128,
-                        sw128_desc(st_k(it), Cfg::kChunkBytes, 1024), idesc_acc, it > 0);
+        bwd_issue_split_a(tbase + 384, tbase + s * 128,
+                          sw128_desc(st_k(it), Cfg::kChunkBytes, 1024), idesc_acc, it > 0);
         tc_commit(k_empty + it % KS);
       }
       if (ok) tc_commit(done);
@@ -817,9 +794,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       tc_fence_after();
       const uint32_t tS = tbase + (it & 1) * 128;  // this block's S buffer
       const bool open = mg.tile_open(q0, kb);  // uniform: the whole tile is unmasked
-      // this half's 64 key columns of S and dP; dS goes to S columns [32 cg, 32 cg +
-      // 32), which hold scores of warpgroup 0: warpgroup 1 stores only once those
-      // are in warpgroup 0's registers
+      // this half's 64 key columns of S and dP; dS (16-bit) goes to S columns
+      // [64 cg, 64 cg + 32), over this warpgroup's own scores
       uint32_t sv[64], dp[64];
       tmem_ld32(tS + cg * 64 + lane_off, sv);
       tmem_ld32(tS + cg * 64 + 32 + lane_off, sv + 32);
@@ -832,11 +808,6 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dp_read);  // dP(j+1) may overwrite the dP columns
-      if (cg == 0) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_read[it & 1]);
-      }
       // every exponential is taken, a masked one then dropped by a select (no
       // branch per element: the loop stays one block the scheduler can overlap)
       uint32_t ps[32];
@@ -865,16 +836,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         grads(std::false_type{});
       else
         grads(std::true_type{});
-      if (cg == 1) {
-        ok = wait_bounded(s_read[it & 1], (it >> 1) & 1, w);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-      }
-      tmem_st16(tS + cg * 32 + lane_off, ps);
-      tmem_st16(tS + cg * 32 + 16 + lane_off, ps + 16);
+      tmem_st16(tS + cg * 64 + lane_off, ps);
+      tmem_st16(tS + cg * 64 + 16 + lane_off, ps + 16);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
