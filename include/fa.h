@@ -70,10 +70,13 @@ enum fa_dtype { FA_FP16 = 0, FA_BF16 = 1, FA_FP32 = 2 /* fa_combine output only 
 enum fa_device_flag {
     FA_DEV_WAIT_TIMEOUT = 1u,   /* a pipeline wait exceeded its time limit; that CTA stopped */
     FA_DEV_BAD_BLOCK = 2u,      /* a block_table entry was outside [0, num_blocks) */
-    FA_DEV_BAD_LENGTH = 4u      /* a cache length (cache_seqlens[b], plus appended keys)
+    FA_DEV_BAD_LENGTH = 4u,     /* a cache length (cache_seqlens[b], plus appended keys)
                                    was negative or beyond the cache's capacity; the
                                    kernel clamped it (attention) or skipped the row
                                    (append) */
+    FA_DEV_SMEM_ALIGN = 8u      /* fa_bwd: the dynamic shared memory did not start on a
+                                   1 KiB boundary, which the dK/dV kernel's layout needs;
+                                   that kernel did nothing and dK, dV are undefined */
 };
 
 /*

@@ -49,34 +49,42 @@ namespace {
 
 constexpr float kBwdLog2e = 1.4426950408889634f;
 
-// Shared memory of the dK/dV kernel: K_j and V_j, a two-stage ring of {Q_i, dO_i}
-// and the column statistics of each stage.
+// Shared memory of the dK/dV kernel: K_j and V_j, a three-stage ring of Q_i, a
+// two-stage ring of dO_i and the column statistics of each dO stage.  Q_i is read
+// by S^T(i), early in a block, and by dK(i), its last product: with three stages the
+// tile two blocks ahead is requested as soon as dK of the block before is done, so
+// it has landed before S^T wants it.  At D = 128 this fills the 227 KiB a CTA may
+// have, with no room left to align the base: the kernel relies on the dynamic shared
+// memory starting on a 1 KiB boundary (it does, at shared address 0x400, measured)
+// and checks it.
 template <int D>
 struct BwdCfg {
   static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms per row
   static constexpr int kTileBytes = 128 * D * 2;      // one 128-row tile
   static constexpr int kChunkBytes = 128 * 128;
+  static constexpr int kQStages = 3, kDoStages = 2;
   static constexpr int kFixA = 0;                     // K_j
   static constexpr int kFixB = kTileBytes;            // V_j
-  static constexpr int kStage = 2 * kTileBytes;       // 2 stages x {Q_i, dO_i}
+  static constexpr int kQ = 2 * kTileBytes;           // Q ring
+  static constexpr int kDo = kQ + kQStages * kTileBytes;  // dO ring
   // column statistics [2 slots][LSE * log2 e | D][kStatPitch] fp32: a tensor copy must
   // start at a column that is a multiple of 4 (16 bytes), so a varlen block whose rows
   // start elsewhere loads from the multiple of 4 below it, kStatLen columns wide, and is
   // read from the remainder on; each copy's destination sits on 128 bytes (the pitch)
   static constexpr int kStatLen = 132;
   static constexpr int kStatPitch = 160;  // 640 bytes: a multiple of 128
-  static constexpr int kStat = kStage + 4 * kTileBytes;
-  static constexpr int kBarOff = kStat + 2 * 2 * kStatPitch * 4;
+  static constexpr int kStat = kDo + kDoStages * kTileBytes;
+  static constexpr int kBarOff = kStat + kDoStages * 2 * kStatPitch * 4;
   static_assert(kStat % 128 == 0 && (kStatPitch * 4) % 128 == 0, "tensor copy destinations");
-  // fix_full, full[2], empty[2], s_full, p_full, done, drain, dp_full, ds_full
-  static constexpr int kNumBars = 11;
+  // fix_full, q_full[3], q_empty[3], do_full[2], do_empty[2], s_full, p_full, done,
+  // drain, dp_full, ds_full
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDoStages + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
-  // room to align the base to 1 KiB; at least 116 KiB, so that one CTA fills an SM
-  // (each takes all 512 tensor-memory columns; a second one would wait in its
-  // allocation for the first to finish)
-  static constexpr int kSmemAlloc =
-      (kSmemBytes + 1024 > 116 * 1024) ? kSmemBytes + 1024 : 116 * 1024;
+  // at least 116 KiB, so that one CTA fills an SM (each takes all 512 tensor-memory
+  // columns; a second one would wait in its allocation for the first to finish)
+  static constexpr int kSmemAlloc = (kSmemBytes > 116 * 1024) ? kSmemBytes : 116 * 1024;
+  static_assert(kSmemAlloc <= 227 * 1024, "dK/dV tiles exceed shared memory");
   static constexpr int kTmemCols = 512;                 // S^T 128 + dP^T 128 + 2 x D
 };
 
@@ -242,9 +250,14 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmD,
                     const BwdParams p) {
   using Cfg = BwdCfg<D>;
+  constexpr int QS = Cfg::kQStages, DS = Cfg::kDoStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // the layout has no slack to align the base: it must already sit on 1 KiB
+  if ((smem_u32(smem_raw) & 1023u) != 0) {  // uniform: nothing set up yet
+    if (threadIdx.x == 0) atomicOr(p.status, kDevSmemAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   // grid: KV heads fastest, key blocks slowest: under a causal mask key block 0
@@ -265,26 +278,34 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 
   uint8_t* fixA = smem + Cfg::kFixA;  // K_j
   uint8_t* fixB = smem + Cfg::kFixB;  // V_j
-  uint8_t* stage = smem + Cfg::kStage;  // slot s: Q_i at s * 2 tiles, dO_i after it
-  float* stat = reinterpret_cast<float*>(smem + Cfg::kStat);  // [slot][lse2 | D][128]
+  uint8_t* q_ring = smem + Cfg::kQ;    // slot n % 3: Q of block n
+  uint8_t* do_ring = smem + Cfg::kDo;  // slot n % 2: dO of block n
+  float* stat = reinterpret_cast<float*>(smem + Cfg::kStat);  // [dO slot][lse2 | D][pitch]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
   uint64_t* fix_full = bars;
-  uint64_t* full = bars + 1;
-  uint64_t* empty = bars + 3;
-  uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* done = bars + 7;
-  uint64_t* drain = bars + 8;
-  uint64_t* dp_full = bars + 9;
-  uint64_t* ds_full = bars + 10;
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = q_full + QS;
+  uint64_t* do_full = q_empty + QS;  // dO and the column statistics
+  uint64_t* do_empty = do_full + DS;
+  uint64_t* s_full = do_empty + DS;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* done = s_full + 2;
+  uint64_t* drain = s_full + 3;
+  uint64_t* dp_full = s_full + 4;
+  uint64_t* ds_full = s_full + 5;
+  static_assert(1 + 2 * QS + 2 * DS + 6 == Cfg::kNumBars, "barrier count");
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
   if (warp == 8 && lane == 0) {
     mbar_init(fix_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(empty + s, 1);
+    for (int s = 0; s < QS; ++s) {
+      mbar_init(q_full + s, 1);
+      mbar_init(q_empty + s, 1);
+    }
+    for (int s = 0; s < DS; ++s) {
+      mbar_init(do_full + s, 1);
+      mbar_init(do_empty + s, 1);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
@@ -321,32 +342,54 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         tma_load_4d(fixA + c * Cfg::kChunkBytes, &tmK, fix_full, c * 64, sq.ks + k0, hk, sq.bc);
         tma_load_4d(fixB + c * Cfg::kChunkBytes, &tmV, fix_full, c * 64, sq.ks + k0, hk, sq.bc);
       }
-      int last[2] = {-1, -1};
+      // the Q stream (the dO stream and the statistics are warp 10's)
+      int last[QS];
+      for (int s = 0; s < QS; ++s) last[s] = -1;
       for (int n = 0; n < n_iter; ++n) {
-        const int s = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
+        const int s = n % QS;
+        const uint32_t ph = (n / QS) & 1;
         const int h = hk * p.G + n / nqb;
         const int qb = (i_lo + n % nqb) * 128;
-        if (!wait_bounded(empty + s, ph ^ 1, w)) break;
-        // Q_i, dO_i and the block's column statistics (LSE * log2 e and D; zero past
-        // the end of the rows, where the mask keeps P at 0)
-        constexpr int kStatBox = VARLEN ? Cfg::kStatLen : 128;  // the tensor maps' box width
-        const int x0 = VARLEN ? ((sq.qs + qb) & ~3) : sq.qs + qb;
-        mbar_arrive_expect_tx(full + s, 2 * Cfg::kTileBytes + 2 * kStatBox * 4);
-        uint8_t* st = stage + s * 2 * Cfg::kTileBytes;
-        for (int c = 0; c < Cfg::kChunks; ++c) {
-          tma_load_4d(st + c * Cfg::kChunkBytes, &tmQ, full + s, c * 64, sq.qs + qb, h, sq.bc);
-          tma_load_4d(st + Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmDO, full + s, c * 64,
-                      sq.qs + qb, h, sq.bc);
-        }
-        tma_load_2d(stat + (2 * s) * Cfg::kStatPitch, &tmL, full + s, x0, sq.bc * p.H + h);
-        tma_load_2d(stat + (2 * s + 1) * Cfg::kStatPitch, &tmD, full + s, x0, sq.bc * p.H + h);
+        if (!wait_bounded(q_empty + s, ph ^ 1, w)) break;
+        mbar_arrive_expect_tx(q_full + s, Cfg::kTileBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_4d(q_ring + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmQ, q_full + s,
+                      c * 64, sq.qs + qb, h, sq.bc);
         last[s] = ph;
       }
       if (*abort_flag) {  // let this CTA's own copies land before the smem goes away
         wait_drain_bwd(fix_full, 0, p.timeout_ns);
-        for (int s = 0; s < 2; ++s)
-          if (last[s] >= 0) wait_drain_bwd(full + s, last[s], p.timeout_ns);
+        for (int s = 0; s < QS; ++s)
+          if (last[s] >= 0) wait_drain_bwd(q_full + s, last[s], p.timeout_ns);
+      }
+    }
+    __syncwarp();
+   } else if (warp == 10) {
+    // ======================================================== TMA producer: dO
+    if (lane == 0 && n_iter > 0) {
+      int last[DS];
+      for (int s = 0; s < DS; ++s) last[s] = -1;
+      for (int n = 0; n < n_iter; ++n) {
+        const int s = n % DS;
+        const uint32_t ph = (n / DS) & 1;
+        const int h = hk * p.G + n / nqb;
+        const int qb = (i_lo + n % nqb) * 128;
+        if (!wait_bounded(do_empty + s, ph ^ 1, w)) break;
+        // dO_i and the block's column statistics (LSE * log2 e and D; zero past the
+        // end of the rows, where the mask keeps P at 0)
+        constexpr int kStatBox = VARLEN ? Cfg::kStatLen : 128;  // the tensor maps' box width
+        const int x0 = VARLEN ? ((sq.qs + qb) & ~3) : sq.qs + qb;
+        mbar_arrive_expect_tx(do_full + s, Cfg::kTileBytes + 2 * kStatBox * 4);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_4d(do_ring + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tmDO, do_full + s,
+                      c * 64, sq.qs + qb, h, sq.bc);
+        tma_load_2d(stat + (2 * s) * Cfg::kStatPitch, &tmL, do_full + s, x0, sq.bc * p.H + h);
+        tma_load_2d(stat + (2 * s + 1) * Cfg::kStatPitch, &tmD, do_full + s, x0, sq.bc * p.H + h);
+        last[s] = ph;
+      }
+      if (*abort_flag) {
+        for (int s = 0; s < DS; ++s)
+          if (last[s] >= 0) wait_drain_bwd(do_full + s, last[s], p.timeout_ns);
       }
     }
     __syncwarp();
@@ -364,40 +407,46 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       // P^T(n+1) overlaps dK(n) and dP^T(n+1).  A product that overwrites a region
       // (S^T(n+1) over P^T(n), dP^T(n+1) over dS^T(n)) is issued after the one
       // reading it, and each commit covers every earlier product of this thread.
-      auto st_q = [&](int s) { return smem_u32(stage + s * 2 * Cfg::kTileBytes); };
-      bool ok = wait_bounded(fix_full, 0, w) && wait_bounded(full, 0, w);
+      auto st_q = [&](int n) { return smem_u32(q_ring + (n % QS) * Cfg::kTileBytes); };
+      auto st_do = [&](int n) { return smem_u32(do_ring + (n % DS) * Cfg::kTileBytes); };
+      bool ok = wait_bounded(fix_full, 0, w) && wait_bounded(q_full, 0, w);
       if (ok) {
         tc_fence_after();
         fwd_issue_qk<D>(tbase, dKk, sw128_desc(st_q(0), 16, 1024), idesc_s);         // S^T(0)
         tc_commit(s_full);
-        fwd_issue_qk<D>(tbase + 128, dVk, sw128_desc(st_q(0) + Cfg::kTileBytes, 16, 1024),
-                        idesc_s);                                                      // dP^T(0)
+        ok = wait_bounded(do_full, 0, w);
+      }
+      if (ok) {
+        tc_fence_after();
+        fwd_issue_qk<D>(tbase + 128, dVk, sw128_desc(st_do(0), 16, 1024), idesc_s);  // dP^T(0)
         tc_commit(dp_full);
       }
       for (int n = 0; n < n_iter && ok; ++n) {
-        const int s = n & 1;
         const bool more = n + 1 < n_iter;
-        const uint32_t sq = st_q(s);
-        const uint32_t sdo = sq + Cfg::kTileBytes;
+        const int n1 = n + 1;
         if (!(ok = wait_bounded(p_full, n & 1, w))) break;
         tc_fence_after();
         // B operands MN-major: rows are queries, the head dim contiguous
-        bwd_issue_split_a(tbase + 256, tbase, sw128_desc(sdo, Cfg::kChunkBytes, 1024), idesc_acc,
-                          n > 0);                                                 // dV(n)
+        bwd_issue_split_a(tbase + 256, tbase, sw128_desc(st_do(n), Cfg::kChunkBytes, 1024),
+                          idesc_acc, n > 0);                                      // dV(n)
         if (more) {
-          if (!(ok = wait_bounded(full + (s ^ 1), ((n + 1) >> 1) & 1, w))) break;
+          if (!(ok = wait_bounded(q_full + n1 % QS, (n1 / QS) & 1, w))) break;
           tc_fence_after();
-          fwd_issue_qk<D>(tbase, dKk, sw128_desc(st_q(s ^ 1), 16, 1024), idesc_s);  // S^T(n+1)
+          fwd_issue_qk<D>(tbase, dKk, sw128_desc(st_q(n1), 16, 1024), idesc_s);      // S^T(n+1)
           tc_commit(s_full);
         }
         if (!(ok = wait_bounded(ds_full, n & 1, w))) break;
         tc_fence_after();
-        bwd_issue_split_a(tbase + 256 + D, tbase + 128, sw128_desc(sq, Cfg::kChunkBytes, 1024),
+        bwd_issue_split_a(tbase + 256 + D, tbase + 128, sw128_desc(st_q(n), Cfg::kChunkBytes, 1024),
                           idesc_acc, n > 0);                                      // dK(n)
-        tc_commit(empty + s);
+        // Q(n) and dO(n) (with the statistics the compute warps read until dS^T(n))
+        // are done with
+        tc_commit(q_empty + n % QS);
+        tc_commit(do_empty + n % DS);
         if (more) {
-          fwd_issue_qk<D>(tbase + 128, dVk,
-                          sw128_desc(st_q(s ^ 1) + Cfg::kTileBytes, 16, 1024), idesc_s);  // dP^T(n+1)
+          if (!(ok = wait_bounded(do_full + n1 % DS, (n1 / DS) & 1, w))) break;
+          tc_fence_after();
+          fwd_issue_qk<D>(tbase + 128, dVk, sw128_desc(st_do(n1), 16, 1024), idesc_s);  // dP^T(n+1)
           tc_commit(dp_full);
         }
       }
@@ -416,12 +465,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
     bool ok = true;
     for (int n = 0; n < n_iter; ++n) {
-      const int s = n & 1;
+      const int s = n % DS;  // the dO slot holding this block's column statistics
       const int h = hk * p.G + n / nqb;
       const int qb = (i_lo + n % nqb) * 128;
       const float slope2 = ALIBI ? p.alibi[h] * kBwdLog2e : 0.f;
-      // the stage (with this block's column statistics) has landed, and S^T is ready
-      ok = wait_bounded(full + s, (n >> 1) & 1, w) && wait_bounded(s_full, n & 1, w);
+      // the block's column statistics have landed, and S^T is ready
+      ok = wait_bounded(do_full + s, (n / DS) & 1, w) && wait_bounded(s_full, n & 1, w);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;

@@ -20,6 +20,7 @@ namespace fa {
 constexpr unsigned kDevWaitTimeout = 1u;  // FA_DEV_WAIT_TIMEOUT
 constexpr unsigned kDevBadBlock = 2u;     // FA_DEV_BAD_BLOCK
 constexpr unsigned kDevBadLength = 4u;    // FA_DEV_BAD_LENGTH
+constexpr unsigned kDevSmemAlign = 8u;    // FA_DEV_SMEM_ALIGN
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
