@@ -117,6 +117,17 @@ def test_alibi_bf16_d64():
              alibi_slopes=synth.alibi_slopes(4))
 
 
+def test_long_gqa_causal_bf16_d128():
+    """Four query heads per KV head over 9 query blocks: the dK/dV kernel streams up to
+    36 (head, query block) iterations through its 3-slot Q and 2-slot dO rings, so every
+    slot and barrier phase comes round many times."""
+    run_case(1, 1100, 1100, 4, 1, 128, torch.bfloat16, 1810, causal=True)
+
+
+def test_long_gqa_window_fp16_d64():
+    run_case(1, 1000, 1000, 8, 2, 64, torch.float16, 1811, window_size=(300, 50))
+
+
 def test_dead_rows_get_zero_dq():
     dq, _, _ = run_case(1, 300, 130, 2, 2, 64, torch.float16, 1804, causal=True)
     assert torch.all(dq[0, :170].float() == 0)
