@@ -260,11 +260,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   uint8_t* smem = smem_raw;
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  // grid: KV heads fastest, key blocks slowest: under a causal mask key block 0
-  // is seen by every query block, so the heaviest CTAs start first
-  const int k0 = blockIdx.z * 128;
-  const int hk = blockIdx.x;
-  const int b = blockIdx.y;
+  // grid: key blocks fastest, then KV heads, then sequences, so the CTAs that
+  // stream one head's query tiles run together and find them in L2; within a
+  // head key block 0 (seen by every query block under a causal mask) starts first
+  const int k0 = blockIdx.x * 128;
+  const int hk = blockIdx.y;
+  const int b = blockIdx.z;
   const BwdSeq sq = bwd_seq<VARLEN>(p, b);
   if (k0 >= sq.Sk) return;  // uniform: past this sequence's keys (varlen), nothing set up yet
   const MaskGeo mg = mask_geo(p, sq.Sq, sq.Sk);
@@ -656,11 +657,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  // grid: heads fastest, query blocks slowest and last first (the last query
-  // block sees the most keys under a causal mask: heaviest CTAs start first)
-  const int q0 = (static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z)) * 128;
-  const int h = blockIdx.x;
-  const int b = blockIdx.y;
+  // grid: query blocks fastest, then heads, then sequences, so the CTAs that
+  // stream one head's key/value tiles run together and find them in L2; within
+  // a head the last query block (the most keys under a causal mask) starts first
+  const int q0 = (static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)) * 128;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
   const int hk = h / p.G;
   const BwdSeq sq = bwd_seq<VARLEN>(p, b);
   if (q0 >= sq.Sq) return;  // uniform: past this sequence's rows (varlen), nothing set up yet
@@ -950,10 +952,10 @@ cudaError_t launch_bwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const 
   if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 DqCfg<D>::kSmemAlloc)) != cudaSuccess)
     return e;
-  const dim3 gkv(p.Hkv, p.B, (p.rows_k + 127) / 128);
+  const dim3 gkv((p.rows_k + 127) / 128, p.Hkv, p.B);
   kkv<<<gkv, kWideThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, tl, td, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const dim3 gq(p.H, p.B, (p.rows_q + 127) / 128);
+  const dim3 gq((p.rows_q + 127) / 128, p.H, p.B);
   kq<<<gq, kWideThreads, DqCfg<D>::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError();
 }
