@@ -163,6 +163,28 @@ __device__ __forceinline__ BwdSeq bwd_seq(const BwdParams& p, int b) {
   return q;
 }
 
+// The CTA's (block, head, sequence) in a grid of gridDim.x blocks x gridDim.y heads
+// x gridDim.z sequences, dispatched in groups of kGridGroup (sequence, head) pairs:
+// blocks slowest inside a group, so the heaviest block of every pair in the group
+// starts first and the grid ends on light blocks, while at most two groups' streamed
+// tiles are live at once and stay in L2.
+constexpr int kGridGroup = 8;
+struct GridPos {
+  int blk, head, seq;
+};
+__device__ __forceinline__ GridPos grid_pos() {
+  const long long nb = gridDim.x;
+  const long long nhs = static_cast<long long>(gridDim.y) * gridDim.z;
+  const long long lin =
+      blockIdx.x + nb * (blockIdx.y + static_cast<long long>(gridDim.y) * blockIdx.z);
+  const long long per = kGridGroup * nb;
+  const long long g = lin / per, r = lin % per;
+  const long long gsz = min(static_cast<long long>(kGridGroup), nhs - g * kGridGroup);
+  const long long hs = g * kGridGroup + r % gsz;
+  return {static_cast<int>(r / gsz), static_cast<int>(hs % gridDim.y),
+          static_cast<int>(hs / gridDim.y)};
+}
+
 // softcap c: x_raw = Q.K; r = 1 / (exp(2 scale x_raw / c) + 1), tanh(scale x_raw / c) =
 // 1 - 2 r, and its derivative factor 1 - tanh^2 = 4 r (1 - r) (no cancellation near
 // saturation).  Returns the score in base-2 units, c log2(e) (1 - 2 r), and g.
@@ -260,12 +282,13 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   uint8_t* smem = smem_raw;
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  // grid: key blocks fastest, then KV heads, then sequences, so the CTAs that
-  // stream one head's query tiles run together and find them in L2; within a
-  // head key block 0 (seen by every query block under a causal mask) starts first
-  const int k0 = blockIdx.x * 128;
-  const int hk = blockIdx.y;
-  const int b = blockIdx.z;
+  // grid: key blocks x KV heads x sequences in groups of (sequence, KV head) pairs
+  // (grid_pos): the CTAs that stream one head's query tiles run together and find
+  // them in L2; key block 0 (seen by every query block under a causal mask) first
+  const GridPos gp = grid_pos();
+  const int k0 = gp.blk * 128;
+  const int hk = gp.head;
+  const int b = gp.seq;
   const BwdSeq sq = bwd_seq<VARLEN>(p, b);
   if (k0 >= sq.Sk) return;  // uniform: past this sequence's keys (varlen), nothing set up yet
   const MaskGeo mg = mask_geo(p, sq.Sq, sq.Sk);
@@ -657,12 +680,13 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  // grid: query blocks fastest, then heads, then sequences, so the CTAs that
-  // stream one head's key/value tiles run together and find them in L2; within
-  // a head the last query block (the most keys under a causal mask) starts first
-  const int q0 = (static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)) * 128;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
+  // grid: query blocks x heads x sequences in groups of (sequence, head) pairs
+  // (grid_pos): the CTAs that stream one head's key/value tiles run together and
+  // find them in L2; the last query block (the most keys under a causal mask) first
+  const GridPos gp = grid_pos();
+  const int q0 = (static_cast<int>(gridDim.x) - 1 - gp.blk) * 128;
+  const int h = gp.head;
+  const int b = gp.seq;
   const int hk = h / p.G;
   const BwdSeq sq = bwd_seq<VARLEN>(p, b);
   if (q0 >= sq.Sq) return;  // uniform: past this sequence's rows (varlen), nothing set up yet
