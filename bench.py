@@ -442,7 +442,7 @@ def run_bwd(args, rank, world, local):
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": tflops_peak,
                          "unit": "TFLOP/s", "frac": round(achieved / tflops_peak, 4),
                          "traffic": None,
-                         "kernel": "bwd_dot_kernel + bwd_dkdv_kernel + bwd_dq_kernel <128, bf16>",
+                         "kernel": "bwd_dot_kernel + bwd_tiles_kernel (dK/dV and dQ CTAs) <128, bf16>",
                          "peak_source": peak_src},
             "gpu_launches": 3 * K, "clocks": clk.summary()}
 

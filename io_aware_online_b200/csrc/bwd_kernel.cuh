@@ -10,27 +10,29 @@
 // Varlen batches (section 3.2) run each packed sequence as its own problem: a
 // CTA reads its sequence's offsets from cu_seqlens and masks the rows of the
 // neighbouring sequences that its tiles reach.
-// Three kernels, all deterministic (no atomics):
+// Two kernels, all deterministic (no atomics): bwd_dot_kernel, then bwd_tiles_kernel,
+// whose grid holds the dK/dV CTAs followed by the dQ CTAs.
 //   bwd_dot_kernel   D for every query row (one warp per row).
-//   bwd_dkdv_kernel  one CTA per (128-key block, KV head): K_j and V_j stay in
+//   dK/dV CTAs       one CTA per (128-key block, KV head): K_j and V_j stay in
 //                    shared memory while the query blocks (of every query head
 //                    reading this KV head) stream past; per block
 //                      S^T = K_j Q_i^T, dP^T = V_j dO_i^T   (tcgen05, SS)
 //                      P^T, dS^T in registers -> 16-bit in tensor memory
 //                      dV += P^T dO_i, dK += dS^T Q_i        (tcgen05, TS)
 //                    with dV and dK accumulated in tensor memory.
-//   bwd_dq_kernel    one CTA per (128-query block, head): Q_i and dO_i stay in
+//   dQ CTAs          one CTA per (128-query block, head): Q_i and dO_i stay in
 //                    shared memory while the key blocks stream past; per block
 //                      S = Q_i K_j^T, dP = dO_i V_j^T, dS -> 16-bit,
 //                      dQ += dS K_j                           (tcgen05)
 // Roles per CTA (384 threads): warps 0-7 compute in two warpgroups that split
 // each block's columns (thread r of a warpgroup owns tensor-memory lane r: a key
-// row in dK/dV, a query row in dQ), warp 8 TMA producer, warp 9 MMA issuer (one
-// elected thread; it also allocates tensor memory), warps 10-11 idle.  Tensor
-// memory of the dK/dV kernel: S^T [0,128), dP^T [128,256), dV and dK from 256; P^T
-// and dS^T are written as 16-bit pairs over the first 64 columns of S^T and dP^T
-// once those scores are in registers (warpgroup 1 waits for warpgroup 0's read).
-// The dQ kernel's layout is given above it.  Every wait is bounded.
+// row in dK/dV, a query row in dQ), warp 8 TMA producer (K, V and the Q stream in
+// dK/dV; Q, dO and the K/V streams in dQ), warp 9 MMA issuer (one elected thread;
+// it also allocates tensor memory), warp 10 the dO and statistics stream of dK/dV,
+// warp 11 idle.  Tensor memory of a dK/dV CTA: S^T [0,128), dP^T [128,256), dV and
+// dK from 256; each warpgroup writes its P^T and dS^T as 16-bit pairs over its own
+// score columns [64 c, 64 c + 32) once those scores are in registers.  The dQ CTA's
+// layout is given above it.  Every wait is bounded.
 // Included by bwd.cu (dense batches) and bwd_varlen.cu (packed sequences), which
 // compile in parallel.
 #pragma once
@@ -163,26 +165,22 @@ __device__ __forceinline__ BwdSeq bwd_seq(const BwdParams& p, int b) {
   return q;
 }
 
-// The CTA's (block, head, sequence) in a grid of gridDim.x blocks x gridDim.y heads
-// x gridDim.z sequences, dispatched in groups of kGridGroup (sequence, head) pairs:
-// blocks slowest inside a group, so the heaviest block of every pair in the group
-// starts first and the grid ends on light blocks, while at most two groups' streamed
-// tiles are live at once and stay in L2.
+// A CTA's (block, head, sequence) from its index lin in a grid of nb blocks x nh heads
+// x ns sequences, dispatched in groups of kGridGroup (sequence, head) pairs: blocks
+// slowest inside a group, so the heaviest block of every pair in the group starts
+// first and the grid ends on light blocks, while at most two groups' streamed tiles
+// are live at once and stay in L2.
 constexpr int kGridGroup = 8;
 struct GridPos {
   int blk, head, seq;
 };
-__device__ __forceinline__ GridPos grid_pos() {
-  const long long nb = gridDim.x;
-  const long long nhs = static_cast<long long>(gridDim.y) * gridDim.z;
-  const long long lin =
-      blockIdx.x + nb * (blockIdx.y + static_cast<long long>(gridDim.y) * blockIdx.z);
-  const long long per = kGridGroup * nb;
+__device__ __forceinline__ GridPos grid_pos(long long lin, int nb, int nh, int ns) {
+  const long long nhs = static_cast<long long>(nh) * ns;
+  const long long per = static_cast<long long>(kGridGroup) * nb;
   const long long g = lin / per, r = lin % per;
   const long long gsz = min(static_cast<long long>(kGridGroup), nhs - g * kGridGroup);
   const long long hs = g * kGridGroup + r % gsz;
-  return {static_cast<int>(r / gsz), static_cast<int>(hs % gridDim.y),
-          static_cast<int>(hs / gridDim.y)};
+  return {static_cast<int>(r / gsz), static_cast<int>(hs % nh), static_cast<int>(hs / nh)};
 }
 
 // softcap c: x_raw = Q.K; r = 1 / (exp(2 scale x_raw / c) + 1), tanh(scale x_raw / c) =
@@ -240,9 +238,9 @@ __global__ void __launch_bounds__(256) bwd_dot_kernel(const BwdParams p) {
   }
 }
 
-// Both tile kernels run 384 threads: two compute warpgroups (warpgroup c takes
+// Both tile passes run 384 threads: two compute warpgroups (warpgroup c takes
 // columns [64 c, 64 c + 64) of every 128 x 128 block for the block's 128 rows),
-// warp 8 TMA producer, warp 9 MMA issuer, warps 10-11 idle.
+// producer warps 8 (and 10 in dK/dV), warp 9 MMA issuer, the rest idle.
 constexpr int kWideThreads = 384;
 // registers per thread: 168 at launch (one CTA per SM); the compute warpgroups
 // take what the producer, the MMA issuer and the idle warps do not need
@@ -266,11 +264,10 @@ __device__ __forceinline__ void bwd_issue_split_a(uint32_t d_tmem, uint32_t a_tm
 }
 
 template <int D, bool BF16, bool ALIBI, bool SOFTCAP, bool VARLEN>
-__global__ void __launch_bounds__(kWideThreads, 1)
-    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmD,
-                    const BwdParams p) {
+__device__ __forceinline__ void bwd_dkdv_cta(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                             const CUtensorMap& tmV, const CUtensorMap& tmDO,
+                                             const CUtensorMap& tmL, const CUtensorMap& tmD,
+                                             const BwdParams& p, long long lin) {
   using Cfg = BwdCfg<D>;
   constexpr int QS = Cfg::kQStages, DS = Cfg::kDoStages;
   extern __shared__ uint8_t smem_raw[];
@@ -285,7 +282,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   // grid: key blocks x KV heads x sequences in groups of (sequence, KV head) pairs
   // (grid_pos): the CTAs that stream one head's query tiles run together and find
   // them in L2; key block 0 (seen by every query block under a causal mask) first
-  const GridPos gp = grid_pos();
+  const GridPos gp = grid_pos(lin, (p.rows_k + 127) / 128, p.Hkv, p.B);
   const int k0 = gp.blk * 128;
   const int hk = gp.head;
   const int b = gp.seq;
@@ -670,10 +667,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 // once dS(j) is written, dQ(j).  The math of block j overlaps the products of block
 // j+1, and no completion barrier runs two phases ahead of its waiters.
 template <int D, bool BF16, bool ALIBI, bool SOFTCAP, bool VARLEN>
-__global__ void __launch_bounds__(kWideThreads, 1)
-    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                  const BwdParams p) {
+__device__ __forceinline__ void bwd_dq_cta(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                           const CUtensorMap& tmV, const CUtensorMap& tmDO,
+                                           const BwdParams& p, long long lin) {
   using Cfg = DqCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -683,8 +679,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   // grid: query blocks x heads x sequences in groups of (sequence, head) pairs
   // (grid_pos): the CTAs that stream one head's key/value tiles run together and
   // find them in L2; the last query block (the most keys under a causal mask) first
-  const GridPos gp = grid_pos();
-  const int q0 = (static_cast<int>(gridDim.x) - 1 - gp.blk) * 128;
+  const int nqb = (p.rows_q + 127) / 128;
+  const GridPos gp = grid_pos(lin, nqb, p.H, p.B);
+  const int q0 = (nqb - 1 - gp.blk) * 128;
   const int h = gp.head;
   const int b = gp.seq;
   const int hk = h / p.G;
@@ -957,30 +954,47 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   }
 }
 
+// Both tile passes in one grid: CTAs [0, n_kv) are dK/dV CTAs, the rest dQ CTAs.
+// The two passes are independent (each reads only the inputs and D), so dQ CTAs
+// start on the SMs that the last dK/dV CTAs leave idle, without a second launch.
+template <int D, bool BF16, bool ALIBI, bool SOFTCAP, bool VARLEN>
+__global__ void __launch_bounds__(kWideThreads, 1)
+    bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                     const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmD,
+                     const BwdParams p) {
+  const long long n_kv =
+      static_cast<long long>((p.rows_k + 127) / 128) * p.Hkv * static_cast<long long>(p.B);
+  const long long lin = blockIdx.x;
+  if (lin < n_kv)
+    bwd_dkdv_cta<D, BF16, ALIBI, SOFTCAP, VARLEN>(tmQ, tmK, tmV, tmDO, tmL, tmD, p, lin);
+  else
+    bwd_dq_cta<D, BF16, ALIBI, SOFTCAP, VARLEN>(tmQ, tmK, tmV, tmDO, p, lin - n_kv);
+}
+
 template <int D, bool BF16, bool ALIBI, bool SOFTCAP, bool VARLEN>
 cudaError_t launch_bwd_inst(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tl, const CUtensorMap& td,
                             const BwdParams& p, cudaStream_t stream) {
-  using Cfg = BwdCfg<D>;
+  constexpr int kSmem = BwdCfg<D>::kSmemAlloc > DqCfg<D>::kSmemAlloc ? BwdCfg<D>::kSmemAlloc
+                                                                      : DqCfg<D>::kSmemAlloc;
+  const long long n_kv =
+      static_cast<long long>((p.rows_k + 127) / 128) * p.Hkv * static_cast<long long>(p.B);
+  const long long n_q =
+      static_cast<long long>((p.rows_q + 127) / 128) * p.H * static_cast<long long>(p.B);
+  if (n_kv + n_q > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const int64_t rows = static_cast<int64_t>(p.cu_q != nullptr ? 1 : p.B) * p.Sq * p.H;
   constexpr int kRowsPerBlock = 8 * (32 / (D / 8));
   bwd_dot_kernel<D, BF16><<<static_cast<unsigned>((rows + kRowsPerBlock - 1) / kRowsPerBlock), 256,
                             0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  auto kkv = bwd_dkdv_kernel<D, BF16, ALIBI, SOFTCAP, VARLEN>;
-  auto kq = bwd_dq_kernel<D, BF16, ALIBI, SOFTCAP, VARLEN>;
-  if ((e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Cfg::kSmemAlloc)) != cudaSuccess)
+  auto kt = bwd_tiles_kernel<D, BF16, ALIBI, SOFTCAP, VARLEN>;
+  if ((e = cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem)) !=
+      cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                DqCfg<D>::kSmemAlloc)) != cudaSuccess)
-    return e;
-  const dim3 gkv((p.rows_k + 127) / 128, p.Hkv, p.B);
-  kkv<<<gkv, kWideThreads, Cfg::kSmemAlloc, stream>>>(tq, tk, tv, tdo, tl, td, p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const dim3 gq((p.rows_q + 127) / 128, p.H, p.B);
-  kq<<<gq, kWideThreads, DqCfg<D>::kSmemAlloc, stream>>>(tq, tk, tv, tdo, p);
+  kt<<<static_cast<unsigned>(n_kv + n_q), kWideThreads, kSmem, stream>>>(tq, tk, tv, tdo, tl, td,
+                                                                        p);
   return cudaGetLastError();
 }
 
