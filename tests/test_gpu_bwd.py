@@ -128,6 +128,13 @@ def test_long_gqa_window_fp16_d64():
     run_case(1, 1000, 1000, 8, 2, 64, torch.float16, 1811, window_size=(300, 50))
 
 
+def test_grid_groups_end_ragged_fp16_d64():
+    """Nine (sequence, KV head) pairs for the dK/dV CTAs and eighteen (sequence, head)
+    pairs for the dQ CTAs: the grid's groups of eight pairs end on a partial group in
+    both passes, with three blocks per pair."""
+    run_case(3, 300, 300, 6, 3, 64, torch.float16, 1812, causal=True)
+
+
 def test_dead_rows_get_zero_dq():
     dq, _, _ = run_case(1, 300, 130, 2, 2, 64, torch.float16, 1804, causal=True)
     assert torch.all(dq[0, :170].float() == 0)
