@@ -386,7 +386,7 @@ BWD = dict(B=4, S=4096, H=32, Hkv=32, d=128, dtype="bf16", causal=True)
 
 
 def run_bwd(args, rank, world, local):
-    """--only bwd: time fa_bwd (D pre-pass + dK/dV + dQ kernels).  Algorithmic work:
+    """--only bwd: time fa_bwd (D pre-pass + one launch of dK/dV and dQ CTAs).  Algorithmic work:
     the five products of the backward (S, dP, dV, dK, dQ), 10 d FLOPs per allowed
     (query, key) pair, i.e. 2.5x the forward's."""
     import io_aware_online_b200 as fa
@@ -441,10 +441,16 @@ def run_bwd(args, rank, world, local):
                        "untimed)", "parallelism": f"dp{world} (independent replicas)"},
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": tflops_peak,
                          "unit": "TFLOP/s", "frac": round(achieved / tflops_peak, 4),
-                         "traffic": None,
+                         # DRAM bytes of a whole step (both launches), like `achieved`
+                         "traffic": (profiled_traffic("bwd_kernels_causal_B4_S4096_d128.md",
+                                                      ["bwd_kernel.cuh", "bwd.cu", "sm100.cuh",
+                                                       "fa_internal.h"])
+                                     if (c["B"], c["S"], c["H"], c["Hkv"], c["d"]) ==
+                                     (4, 4096, 32, 32, 128) and c["dtype"] == "bf16"
+                                     and c["causal"] else None),
                          "kernel": "bwd_dot_kernel + bwd_tiles_kernel (dK/dV and dQ CTAs) <128, bf16>",
                          "peak_source": peak_src},
-            "gpu_launches": 3 * K, "clocks": clk.summary()}
+            "gpu_launches": 2 * K, "clocks": clk.summary()}  # D pre-pass + tile launch
 
 
 # TFLOPS vs sequence length of the causal prefill (B=4, H=Hkv=32)
